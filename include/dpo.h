@@ -1,0 +1,168 @@
+/*
+ * libdpo: the data-parallel hot path of Direct Preference Optimization (DPO) on
+ * NVIDIA B200 (sm_100a), as a C ABI.
+ *
+ * The path, for a batch of 2B rows (chosen and rejected completions of B
+ * prompts), each row = prompt | completion | pad:
+ *   1. LM-head logits z = h . W^T for every scored position (never stored),
+ *   2. log-softmax over the full vocabulary and the target-token pick,
+ *   3. per-row sum of the completion tokens' log-probabilities, in fp32,
+ *   4. the sigmoid DPO loss from policy and reference sums,
+ *   5. the backward of (4) through (1)-(3) to dH and dW.
+ * ("DPO Training on GPU, in depth", sections "What one DPO step computes",
+ *  "A worked example of the numbers" and the hand-written sequence_logps /
+ *  dpo_step in "A training configuration that fits".)
+ *
+ * Conventions shared by every call
+ *   - Every buffer is owned by the caller. The library allocates no device
+ *     memory; each call that needs scratch takes a caller-provided workspace
+ *     whose size dpo_workspace_size() returns.
+ *   - Device pointers must point to device memory of the current CUDA device.
+ *     "host" marks the few arguments read from host memory during the call.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream). All device
+ *     work is enqueued on it; calls return without waiting for the GPU, except
+ *     dpo_check(), which synchronises the stream.
+ *   - Errors the host can see (bad sizes, null pointers, misalignment, too
+ *     small a workspace, unsupported dtype) are returned before any launch and
+ *     leave every output untouched.
+ *   - Errors only the GPU can see (a target token outside [0, V), a pipeline
+ *     wait that exceeded its time budget) are recorded in a per-device status
+ *     word that dpo_check() reads and clears. A bad target is scored as 0.
+ *   - The forward is deterministic: the same inputs give bit-identical outputs.
+ *
+ * Row model (all calls that take a dpo_batch)
+ *   Row r has prompt length P_r = prompt_len[r] >= 1 and completion length
+ *   C_r = completion_len[r] >= 0 with P_r + C_r <= L. Completion tokens are
+ *   tokens[r, P_r .. P_r + C_r - 1]; token j is predicted by position j - 1, so
+ *   the scored positions are t in [P_r - 1, P_r + C_r - 1) and position t
+ *   scores tokens[r, t + 1] ("DPO Training on GPU, in depth", sequence_logps:
+ *   logits[:, :-1] pair with labels[:, 1:] and mask[:, 1:]). Positions outside
+ *   that range (prompt, pad, the last position) contribute nothing.
+ *   Nc = sum_r C_r is the number of scored positions.
+ */
+#ifndef LIBDPO_DPO_H
+#define LIBDPO_DPO_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  DPO_OK = 0,
+  DPO_ERR_INVALID_ARG = 1,  /* null pointer, size out of range, P_r/C_r do not fit L   */
+  DPO_ERR_UNSUPPORTED = 2,  /* dtype (fp16 is refused), d not a multiple of 8, ...      */
+  DPO_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed                        */
+  DPO_ERR_TIMEOUT = 4,      /* device: a pipeline wait ran out of its time budget       */
+  DPO_ERR_BAD_TARGET = 5,   /* device: a scored target token was outside [0, V)         */
+  DPO_ERR_WORKSPACE = 6     /* workspace null, too small or not 256-byte aligned        */
+} dpo_status;
+
+/* Element type of H and W. fp16 is refused: the pages' recipe raises on full
+ * fp16 training because log-prob ratios leave fp16's range ("Run Distributed
+ * Full-Model DPO with PyTorch FSDP", "What to Watch Out For"). DPO_BF16 runs on
+ * the tcgen05 tensor cores with fp32 accumulation; DPO_F32 runs an exact-fp32
+ * SIMT path meant for small problems. */
+typedef enum { DPO_BF16 = 0, DPO_F32 = 1, DPO_F16 = 2 } dpo_dtype;
+
+/* Which rows form pair i. HALVES: chosen row i, rejected row B + i (the
+ * concatenated [2B, L] batch, "Run Distributed Full-Model DPO with PyTorch
+ * FSDP", Step 4). ADJACENT: chosen row 2i, rejected row 2i + 1 (pairs next to
+ * each other in the micro batch, Megatron-Bridge PR 6092 changelog). */
+typedef enum { DPO_PAIRS_HALVES = 0, DPO_PAIRS_ADJACENT = 1 } dpo_layout;
+
+typedef struct {
+  int32_t R;                     /* rows (2B for a preference batch), 1 <= R <= 65535  */
+  int32_t L;                     /* positions per row, 2 <= L                           */
+  int32_t d;                     /* hidden size; a multiple of 8, 8 <= d <= 65536       */
+  int32_t V;                     /* vocabulary size, 1 <= V <= 2^24                     */
+  int32_t dtype;                 /* dpo_dtype of H and W                                */
+  const void* H;                 /* device [R, L, d] row-major hidden states (LM-head
+                                    input); 16-byte aligned                             */
+  const void* W;                 /* device [V, d] row-major LM-head weight (policy or
+                                    reference), logits = H . W^T; 16-byte aligned       */
+  const int32_t* tokens;         /* device [R, L] token ids                             */
+  const int32_t* prompt_len;     /* host [R], P_r >= 1                                  */
+  const int32_t* completion_len; /* host [R], C_r >= 0, P_r + C_r <= L                  */
+} dpo_batch;
+
+/* Workspace bytes that dpo_seq_logprobs (fwd_bytes) and dpo_backward
+ * (bwd_bytes) need for this batch. Either output pointer may be NULL.
+ * bwd_bytes is the size that lets the backward run in one token chunk; a
+ * smaller workspace of at least *bwd_min_bytes (may be NULL) makes it run in
+ * several chunks. Pure host function. */
+dpo_status dpo_workspace_size(const dpo_batch* batch, size_t* fwd_bytes, size_t* bwd_bytes,
+                              size_t* bwd_min_bytes);
+
+/* Per-row completion log-prob sums (steps 1-3), for the policy or the
+ * reference, with or without what the backward needs.
+ *   seq_logp  device [R] fp32, out: S_r = sum over scored t of log p(tokens[r,t+1])
+ *   tok_logp  device [R, L] fp32 or NULL, out: log p at scored positions, 0 elsewhere
+ *   lse_state device [Nc] fp32, out: log-sum-exp of each scored position in row
+ *             order; required when want_grad != 0 (dpo_backward reads it), else
+ *             may be NULL
+ *   ws        device workspace of ws_bytes >= fwd_bytes, 256-byte aligned
+ * Sums carry no beta, so one scoring pass serves every beta (offline reference
+ * scoring: Megatron-Bridge PR 6092, "Why the reference is scored offline"); rows
+ * keep their order so stored sums can be joined back by row index. */
+dpo_status dpo_seq_logprobs(const dpo_batch* batch, int want_grad, float* seq_logp,
+                            float* tok_logp, float* lse_state, void* ws, size_t ws_bytes,
+                            void* stream);
+
+/* Sigmoid DPO loss and its metrics (step 4), for B pairs.
+ *   pol, ref        device [2B] fp32 sequence sums of policy and reference, in `layout`
+ *   beta            the DPO temperature (> 0)
+ *   grad_scale      factor folded into row_coef (e.g. 1/accumulation steps)
+ *   loss            device [1]: mean over pairs of -log sigmoid(margin)
+ *   accuracy        device [1]: fraction of pairs with margin > 0 (strict)
+ *   margins         device [B]: beta * ((pol_c - ref_c) - (pol_r - ref_r))
+ *   chosen_rewards  device [B]: beta * (pol_c - ref_c)
+ *   rejected_rewards device [B]: beta * (pol_r - ref_r)
+ *   weights         device [B]: sigmoid(-margin), the per-pair gradient weight
+ *   row_coef        device [2B] or NULL: d(grad_scale * loss) / d pol[row]
+ * ("DPO Training on GPU, in depth": the loss formula, the worked example's
+ *  rewards, margin and sigmoid(-margin) weight, and dpo_step's mean loss and
+ *  reward accuracy.) Computed in fp64 on the device, stored as fp32. Any of the
+ * outputs except loss may be NULL. */
+dpo_status dpo_loss(int32_t B, int32_t layout, const float* pol, const float* ref, float beta,
+                    float grad_scale, float* loss, float* accuracy, float* margins,
+                    float* chosen_rewards, float* rejected_rewards, float* weights,
+                    float* row_coef, void* stream);
+
+/* Backward of sum_r row_coef[r] * seq_logp[r] (step 5) to H and W.
+ *   lse_state   device [Nc] fp32 from dpo_seq_logprobs(want_grad=1) on the same batch
+ *   row_coef    device [R] fp32, d(objective)/d seq_logp[r] (dpo_loss writes it)
+ *   dH          device [R, L, d] fp32, out: fully written; 0 at unscored positions
+ *   dW          device [V, d] fp32, out: dW = sum_t dz_t^T h_t, or dW += that when
+ *               accumulate_dW != 0 (gradient accumulation over micro-batches)
+ *   ws          device workspace, >= bwd_min_bytes, 256-byte aligned
+ * with dz[t, v] = row_coef[r(t)] * (1[v = tokens[r, t+1]] - softmax(z_t)[v]). The
+ * logits are recomputed tile by tile. dH may be NULL (only dW is formed). */
+dpo_status dpo_backward(const dpo_batch* batch, const float* lse_state, const float* row_coef,
+                        float* dH, float* dW, int accumulate_dW, void* ws, size_t ws_bytes,
+                        void* stream);
+
+/* Synchronise `stream`, then return and clear the current device's status word
+ * (DPO_OK, DPO_ERR_TIMEOUT or DPO_ERR_BAD_TARGET), or DPO_ERR_CUDA if the
+ * synchronisation itself failed. */
+dpo_status dpo_check(void* stream);
+
+/* Time budget, in milliseconds, of every bounded wait inside the kernels of the
+ * calling host thread's current device (default 4000). A wait that exceeds it
+ * makes the kernel record DPO_ERR_TIMEOUT, drain its in-flight copies and MMAs
+ * (again bounded) and exit. Returns the previous value. */
+uint32_t dpo_set_wait_budget_ms(uint32_t ms);
+
+/* Static description of a status code. */
+const char* dpo_status_string(dpo_status s);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+int32_t dpo_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LIBDPO_DPO_H */

@@ -1,0 +1,389 @@
+// C ABI of libdpo: argument checks, the per-call schedule (packed scored
+// positions), workspace layout, TMA tensor maps and the launch sequence of each
+// entry point. See include/dpo.h for the contract of every call.
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include <cudaTypedefs.h>
+
+#include "dpo.h"
+#include "internal.h"
+
+// Per-device status word: kernels record DPO_ERR_TIMEOUT / DPO_ERR_BAD_TARGET
+// here; dpo_check() reads and clears it.
+__device__ int g_dpo_status_word = 0;
+
+namespace {
+
+using namespace dpo;
+
+constexpr size_t kAlign = 256;
+constexpr int kMinChunk = 128;   // smallest backward token chunk
+
+std::atomic<uint32_t> g_budget_ms{4000};
+
+struct DevInfo {
+  bool ready = false;
+  int* status = nullptr;
+  int sms = 0;
+};
+std::mutex g_mu;
+DevInfo g_dev[256];
+
+dpo_status device_info(DevInfo* out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 256) return DPO_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  DevInfo& di = g_dev[dev];
+  if (!di.ready) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_dpo_status_word) != cudaSuccess) return DPO_ERR_CUDA;
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return DPO_ERR_CUDA;
+    di.status = static_cast<int*>(p);
+    di.sms = sms;
+    di.ready = true;
+  }
+  *out = di;
+  return DPO_OK;
+}
+
+DevCtl make_ctl(const DevInfo& di) {
+  DevCtl c;
+  c.status = di.status;
+  c.budget_ns = static_cast<unsigned long long>(g_budget_ms.load()) * 1000000ull;
+  return c;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 tensor map over a row-major [outer, inner] array with 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+              uint32_t box_inner, uint32_t box_outer) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t es[2] = {1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                        strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+struct Plan {
+  int R = 0, L = 0, d = 0, V = 0, dtype = 0;
+  int Nc = 0;
+  std::vector<int> row_start;          // [R + 1]
+  // common prefix of both workspaces
+  size_t off_rs = 0, off_P = 0, off_y = 0, off_dst = 0, off_rowid = 0, off_hp = 0, prefix = 0;
+  // forward suffix
+  int S = 0, ldp = 0;
+  size_t off_part = 0, off_zy = 0, off_lp = 0, fwd_total = 0;
+  // backward suffix
+  size_t off_G = 0, g_row_bytes = 0, bwd_total = 0, bwd_min = 0;
+  long long ldG = 0;
+};
+
+dpo_status make_plan(const dpo_batch* b, Plan* p) {
+  if (b == nullptr) return DPO_ERR_INVALID_ARG;
+  if (b->dtype == DPO_F16) return DPO_ERR_UNSUPPORTED;
+  if (b->dtype != DPO_BF16 && b->dtype != DPO_F32) return DPO_ERR_INVALID_ARG;
+  if (b->R < 1 || b->R > 65535 || b->L < 2 || b->V < 1 || b->V > (1 << 24) || b->d < 1 ||
+      b->d > 65536)
+    return DPO_ERR_INVALID_ARG;
+  if (b->d % 8 != 0) return DPO_ERR_UNSUPPORTED;
+  if (b->H == nullptr || b->W == nullptr || b->tokens == nullptr || b->prompt_len == nullptr ||
+      b->completion_len == nullptr)
+    return DPO_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(b->H) | reinterpret_cast<uintptr_t>(b->W)) % 16 != 0)
+    return DPO_ERR_INVALID_ARG;
+  if (static_cast<long long>(b->R) * b->L > (1ll << 31) - 2) return DPO_ERR_INVALID_ARG;
+  p->R = b->R;
+  p->L = b->L;
+  p->d = b->d;
+  p->V = b->V;
+  p->dtype = b->dtype;
+  p->row_start.assign(b->R + 1, 0);
+  long long nc = 0;
+  for (int r = 0; r < b->R; ++r) {
+    const int P = b->prompt_len[r], C = b->completion_len[r];
+    if (P < 1 || C < 0 || static_cast<long long>(P) + C > b->L) return DPO_ERR_INVALID_ARG;
+    p->row_start[r] = static_cast<int>(nc);
+    nc += C;
+  }
+  if (nc > (1ll << 30)) return DPO_ERR_INVALID_ARG;
+  p->row_start[b->R] = static_cast<int>(nc);
+  p->Nc = static_cast<int>(nc);
+  const size_t Nc = p->Nc;
+  const bool bf16 = b->dtype == DPO_BF16;
+
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o = align_up(o + bytes, kAlign);
+    return at;
+  };
+  p->off_rs = take(sizeof(int) * (b->R + 1));
+  p->off_P = take(sizeof(int) * b->R);
+  p->off_y = take(sizeof(int) * Nc);
+  p->off_dst = take(sizeof(int) * Nc);
+  p->off_rowid = take(sizeof(int) * Nc);
+  p->off_hp = take(bf16 ? Nc * b->d * 2 : 0);
+  p->prefix = o;
+
+  p->S = bf16 ? (b->V + kBN - 1) / kBN : 1;
+  p->ldp = static_cast<int>(align_up(Nc > 0 ? Nc : 1, 64));
+  p->off_part = take(sizeof(float2) * static_cast<size_t>(p->S) * p->ldp);
+  p->off_zy = take(sizeof(float) * p->ldp);
+  p->off_lp = take(sizeof(float) * p->ldp);
+  p->fwd_total = o;
+
+  o = p->prefix;
+  p->ldG = bf16 ? static_cast<long long>(align_up(b->V, 8)) : b->V;
+  p->g_row_bytes = static_cast<size_t>(p->ldG) * (bf16 ? 2 : 4);
+  p->off_G = o;
+  const size_t full_rows = Nc > 0 ? Nc : 1;
+  const size_t min_rows = full_rows < static_cast<size_t>(kMinChunk) ? full_rows : kMinChunk;
+  p->bwd_total = align_up(o + full_rows * p->g_row_bytes, kAlign);
+  p->bwd_min = align_up(o + min_rows * p->g_row_bytes, kAlign);
+  return DPO_OK;
+}
+
+Sched sched_of(const Plan& p, void* ws) {
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  Sched s;
+  s.row_start = reinterpret_cast<const int*>(w + p.off_rs);
+  s.prompt = reinterpret_cast<const int*>(w + p.off_P);
+  s.y = reinterpret_cast<int*>(w + p.off_y);
+  s.dst = reinterpret_cast<int*>(w + p.off_dst);
+  s.rowid = reinterpret_cast<int*>(w + p.off_rowid);
+  return s;
+}
+
+dpo_status cuda_status(cudaError_t e) { return e == cudaSuccess ? DPO_OK : DPO_ERR_CUDA; }
+
+// Upload the row table and build the scored-position tables (+ packed H for bf16).
+dpo_status stage_schedule(const Plan& p, const dpo_batch* b, void* ws, const DevCtl& ctl,
+                          cudaStream_t st) {
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  std::vector<RowChunk> chunks((p.R + kRowChunk - 1) / kRowChunk);
+  for (size_t c = 0; c < chunks.size(); ++c) {
+    RowChunk& rc = chunks[c];
+    rc.row0 = static_cast<int>(c) * kRowChunk;
+    rc.n = std::min(kRowChunk, p.R - rc.row0);
+    rc.R = p.R;
+    rc.total = p.Nc;
+    for (int i = 0; i < rc.n; ++i) {
+      rc.rs[i] = p.row_start[rc.row0 + i];
+      rc.P[i] = b->prompt_len[rc.row0 + i];
+    }
+    cudaError_t e = launch_upload_rows(rc, reinterpret_cast<int*>(w + p.off_rs),
+                                       reinterpret_cast<int*>(w + p.off_P), st);
+    if (e != cudaSuccess) return DPO_ERR_CUDA;
+  }
+  uint16_t* Hp = p.dtype == DPO_BF16 ? reinterpret_cast<uint16_t*>(w + p.off_hp) : nullptr;
+  return cuda_status(launch_prep(static_cast<const uint16_t*>(b->H), b->tokens, sched_of(p, ws),
+                                 p.R, p.L, p.d, p.V, p.Nc, Hp, ctl, st));
+}
+
+bool ws_ok(const void* ws, size_t have, size_t need) {
+  return ws != nullptr && have >= need && reinterpret_cast<uintptr_t>(ws) % kAlign == 0;
+}
+
+}  // namespace
+
+extern "C" {
+
+dpo_status dpo_workspace_size(const dpo_batch* batch, size_t* fwd_bytes, size_t* bwd_bytes,
+                              size_t* bwd_min_bytes) {
+  Plan p;
+  const dpo_status s = make_plan(batch, &p);
+  if (s != DPO_OK) return s;
+  if (fwd_bytes) *fwd_bytes = p.fwd_total;
+  if (bwd_bytes) *bwd_bytes = p.bwd_total;
+  if (bwd_min_bytes) *bwd_min_bytes = p.bwd_min;
+  return DPO_OK;
+}
+
+dpo_status dpo_seq_logprobs(const dpo_batch* batch, int want_grad, float* seq_logp,
+                            float* tok_logp, float* lse_state, void* ws, size_t ws_bytes,
+                            void* stream) {
+  Plan p;
+  dpo_status s = make_plan(batch, &p);
+  if (s != DPO_OK) return s;
+  if (seq_logp == nullptr || (want_grad && lse_state == nullptr)) return DPO_ERR_INVALID_ARG;
+  if (!ws_ok(ws, ws_bytes, p.fwd_total)) return DPO_ERR_WORKSPACE;
+  DevInfo di;
+  if ((s = device_info(&di)) != DPO_OK) return s;
+  const DevCtl ctl = make_ctl(di);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+
+  if ((s = stage_schedule(p, batch, ws, ctl, st)) != DPO_OK) return s;
+  const Sched sc = sched_of(p, ws);
+  float2* part = reinterpret_cast<float2*>(w + p.off_part);
+  float* zy = reinterpret_cast<float*>(w + p.off_zy);
+  float* lp = reinterpret_cast<float*>(w + p.off_lp);
+
+  if (p.Nc > 0) {
+    if (p.dtype == DPO_BF16) {
+      CUtensorMap mA, mB;
+      if (!make_map(&mA, w + p.off_hp, p.d, p.Nc, 2ull * p.d, kBK, kBM) ||
+          !make_map(&mB, batch->W, p.d, p.V, 2ull * p.d, kBK, kBN))
+        return DPO_ERR_CUDA;
+      if (launch_fwd_lse(mA, mB, p.Nc, p.V, p.d, sc.y, part, p.ldp, zy, di.sms, ctl, st) !=
+          cudaSuccess)
+        return DPO_ERR_CUDA;
+    } else {
+      if (launch_f32_fwd(static_cast<const float*>(batch->H), static_cast<const float*>(batch->W),
+                         sc, p.Nc, p.d, p.V, part, zy, st) != cudaSuccess)
+        return DPO_ERR_CUDA;
+    }
+    if (launch_combine(part, p.ldp, p.S, zy, sc.y, p.Nc, lp, want_grad ? lse_state : nullptr,
+                       st) != cudaSuccess)
+      return DPO_ERR_CUDA;
+  }
+  return cuda_status(launch_rowsum(lp, sc.row_start, sc.prompt, p.R, p.L, seq_logp, tok_logp, st));
+}
+
+dpo_status dpo_loss(int32_t B, int32_t layout, const float* pol, const float* ref, float beta,
+                    float grad_scale, float* loss, float* accuracy, float* margins,
+                    float* chosen_rewards, float* rejected_rewards, float* weights,
+                    float* row_coef, void* stream) {
+  if (B < 1 || B > (1 << 28) || (layout != DPO_PAIRS_HALVES && layout != DPO_PAIRS_ADJACENT))
+    return DPO_ERR_INVALID_ARG;
+  if (pol == nullptr || ref == nullptr || loss == nullptr) return DPO_ERR_INVALID_ARG;
+  if (!(beta > 0.f) || !std::isfinite(beta) || !std::isfinite(grad_scale))
+    return DPO_ERR_INVALID_ARG;
+  return cuda_status(launch_loss(B, layout, pol, ref, beta, grad_scale, loss, accuracy, margins,
+                                 chosen_rewards, rejected_rewards, weights, row_coef,
+                                 static_cast<cudaStream_t>(stream)));
+}
+
+dpo_status dpo_backward(const dpo_batch* batch, const float* lse_state, const float* row_coef,
+                        float* dH, float* dW, int accumulate_dW, void* ws, size_t ws_bytes,
+                        void* stream) {
+  Plan p;
+  dpo_status s = make_plan(batch, &p);
+  if (s != DPO_OK) return s;
+  if ((p.Nc > 0 && lse_state == nullptr) || row_coef == nullptr || dW == nullptr)
+    return DPO_ERR_INVALID_ARG;
+  if (!ws_ok(ws, ws_bytes, p.bwd_min)) return DPO_ERR_WORKSPACE;
+  DevInfo di;
+  if ((s = device_info(&di)) != DPO_OK) return s;
+  const DevCtl ctl = make_ctl(di);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+
+  // Token chunk that fits the workspace (a multiple of 128 unless it covers all).
+  size_t rows_fit = (ws_bytes - p.off_G) / p.g_row_bytes;
+  int Mc = static_cast<int>(std::min<size_t>(rows_fit, static_cast<size_t>(p.Nc)));
+  if (Mc < p.Nc) Mc = Mc / kMinChunk * kMinChunk;
+  if (p.Nc > 0 && Mc < 1) return DPO_ERR_WORKSPACE;
+
+  if ((s = stage_schedule(p, batch, ws, ctl, st)) != DPO_OK) return s;
+  const Sched sc = sched_of(p, ws);
+  if (dH != nullptr &&
+      cudaMemsetAsync(dH, 0, sizeof(float) * static_cast<size_t>(p.R) * p.L * p.d, st) !=
+          cudaSuccess)
+    return DPO_ERR_CUDA;
+  if (p.Nc == 0) {
+    if (!accumulate_dW &&
+        cudaMemsetAsync(dW, 0, sizeof(float) * static_cast<size_t>(p.V) * p.d, st) != cudaSuccess)
+      return DPO_ERR_CUDA;
+    return DPO_OK;
+  }
+  const bool bf16 = p.dtype == DPO_BF16;
+  const uint16_t* Hp = reinterpret_cast<const uint16_t*>(w + p.off_hp);
+  for (int tok0 = 0; tok0 < p.Nc; tok0 += Mc) {
+    const int mc = std::min(Mc, p.Nc - tok0);
+    const int acc = (accumulate_dW || tok0 > 0) ? 1 : 0;
+    if (bf16) {
+      uint16_t* G = reinterpret_cast<uint16_t*>(w + p.off_G);
+      const uint16_t* hp0 = Hp + static_cast<size_t>(tok0) * p.d;
+      CUtensorMap mHk, mWk, mGk, mWmn, mGmn, mHmn;
+      if (!make_map(&mHk, hp0, p.d, mc, 2ull * p.d, kBK, kBM) ||
+          !make_map(&mWk, batch->W, p.d, p.V, 2ull * p.d, kBK, kBN) ||
+          !make_map(&mGk, G, p.V, mc, 2ull * p.ldG, kBK, kBM) ||
+          !make_map(&mWmn, batch->W, p.d, p.V, 2ull * p.d, 64, kBK) ||
+          !make_map(&mGmn, G, p.V, mc, 2ull * p.ldG, 64, kBK) ||
+          !make_map(&mHmn, hp0, p.d, mc, 2ull * p.d, 64, kBK))
+        return DPO_ERR_CUDA;
+      if (launch_bwd_grad(mHk, mWk, mc, p.V, p.d, tok0, sc.y, lse_state, row_coef, sc.rowid, G,
+                          p.ldG, di.sms, ctl, st) != cudaSuccess)
+        return DPO_ERR_CUDA;
+      if (dH != nullptr &&
+          launch_bwd_dh(mGk, mWmn, mc, p.V, p.d, tok0, sc.dst, dH, di.sms, ctl, st) != cudaSuccess)
+        return DPO_ERR_CUDA;
+      if (launch_bwd_dw(mGmn, mHmn, mc, p.V, p.d, dW, acc, di.sms, ctl, st) != cudaSuccess)
+        return DPO_ERR_CUDA;
+    } else {
+      float* G = reinterpret_cast<float*>(w + p.off_G);
+      const float* H = static_cast<const float*>(batch->H);
+      const float* W = static_cast<const float*>(batch->W);
+      if (launch_f32_grad(H, W, sc, tok0, mc, p.d, p.V, lse_state, row_coef, G, st) !=
+          cudaSuccess)
+        return DPO_ERR_CUDA;
+      if (dH != nullptr && launch_f32_dh(G, W, sc, tok0, mc, p.d, p.V, dH, st) != cudaSuccess)
+        return DPO_ERR_CUDA;
+      if (launch_f32_dw(G, H, sc, tok0, mc, p.d, p.V, dW, acc, st) != cudaSuccess)
+        return DPO_ERR_CUDA;
+    }
+  }
+  return DPO_OK;
+}
+
+dpo_status dpo_check(void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  DevInfo di;
+  dpo_status s = device_info(&di);
+  if (s != DPO_OK) return s;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return DPO_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyAsync(&v, di.status, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaMemsetAsync(di.status, 0, sizeof(int), st) != cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess)
+    return DPO_ERR_CUDA;
+  return static_cast<dpo_status>(v);
+}
+
+uint32_t dpo_set_wait_budget_ms(uint32_t ms) { return g_budget_ms.exchange(ms < 1 ? 1 : ms); }
+
+const char* dpo_status_string(dpo_status s) {
+  switch (s) {
+    case DPO_OK: return "ok";
+    case DPO_ERR_INVALID_ARG: return "invalid argument";
+    case DPO_ERR_UNSUPPORTED: return "unsupported (dtype or shape)";
+    case DPO_ERR_CUDA: return "CUDA error";
+    case DPO_ERR_TIMEOUT: return "device wait exceeded its time budget";
+    case DPO_ERR_BAD_TARGET: return "target token outside [0, V)";
+    case DPO_ERR_WORKSPACE: return "workspace missing, too small or misaligned";
+  }
+  return "unknown status";
+}
+
+int32_t dpo_version(void) { return 100; }
+
+}  // extern "C"

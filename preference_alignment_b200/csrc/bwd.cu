@@ -1,0 +1,197 @@
+// Backward kernels of the DPO head path (bf16 tensor-core route).
+//
+// The objective is sum_r coef_r * S_r with S_r the row's completion log-prob sum,
+// so for a scored position t of row r the logit gradient is
+//   dz[t, v] = coef_r * (1[v = y_t] - softmax(z_t)[v])
+// and dH[t] = dz[t] . W, dW = sum_t dz[t]^T h_t (chain rule through log-softmax;
+// the pages run this as loss.backward() on the chunked, checkpointed loss of
+// "DPO Training on GPU, in depth", "A training configuration that fits", which
+// recomputes each chunk's log-softmax in the backward: here the logits are
+// recomputed tile by tile).
+//
+// Three persistent tcgen05 GEMMs per token chunk:
+//   k_tc_gemm<K,K,EpiGrad>  z tile = Hp . W^T, epilogue forms dz in bf16 (never z)
+//   k_tc_gemm<K,MN,EpiRows> dH chunk = dz . W        (K = V)
+//   k_tc_gemm<MN,MN,EpiDW>  dW (+)= dz^T . Hp        (K = tokens)
+#include <cmath>
+
+#include "internal.h"
+#include "tc_gemm.cuh"
+
+namespace dpo {
+
+constexpr float kLog2eB = 1.4426950408889634f;
+
+// ------------------------------------------------------------------ dz epilogue
+struct EpiGrad {
+  struct Params {
+    const int* y;
+    const float* lse;
+    const float* coef;     // [R] per-row coefficient
+    const int* rowid;
+    uint16_t* G;           // [Mc, ldG] bf16 chunk
+    long long ldG;
+    int Mc, V, tok0;
+  };
+  int vbase, yl;
+  bool valid;
+  float nl2, cf;
+  uint16_t* out;
+
+  __device__ __forceinline__ void begin(const Params& p, int mt, int nt, int row) {
+    const int tok = mt * kBM + row;
+    valid = tok < p.Mc;
+    vbase = nt * kBN;
+    yl = -1;
+    nl2 = 0.f;
+    cf = 0.f;
+    out = nullptr;
+    if (valid) {
+      const int gt = p.tok0 + tok;
+      const int y = __ldg(p.y + gt);
+      yl = y - vbase;
+      nl2 = -__ldg(p.lse + gt) * kLog2eB;
+      cf = y >= 0 ? __ldg(p.coef + __ldg(p.rowid + gt)) : 0.f;  // bad target: no gradient
+      out = p.G + static_cast<long long>(tok) * p.ldG + vbase;
+    }
+  }
+
+  __device__ __forceinline__ void chunk(const Params& p, int c, const uint32_t (&v)[32]) {
+    if (!valid) return;
+    uint32_t packed[16];
+#pragma unroll
+    for (int j = 0; j < 32; j += 2) {
+      const int col = c * 32 + j;
+      float g0 = cf * ((col == yl ? 1.f : 0.f) -
+                       ex2_approx(fmaf(__uint_as_float(v[j]), kLog2eB, nl2)));
+      float g1 = cf * ((col + 1 == yl ? 1.f : 0.f) -
+                       ex2_approx(fmaf(__uint_as_float(v[j + 1]), kLog2eB, nl2)));
+      if (vbase + col >= p.V) g0 = 0.f;
+      if (vbase + col + 1 >= p.V) g1 = 0.f;
+      packed[j / 2] = pack_bf16x2(g0, g1);
+    }
+    uint4* dst = reinterpret_cast<uint4*>(out + c * 32);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      if (vbase + c * 32 + q * 8 < p.ldG)
+        dst[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+    }
+  }
+
+  __device__ __forceinline__ void end(const Params&) {}
+};
+
+// ------------------------------------------------------------------ dH rows epilogue
+struct EpiRows {
+  struct Params {
+    const int* dst;        // packed position -> flat row r * L + t
+    float* out;            // dH [R * L, d]
+    int Mc, d, tok0;
+  };
+  float* o;
+  int nbase;
+  bool valid;
+
+  __device__ __forceinline__ void begin(const Params& p, int mt, int nt, int row) {
+    const int tok = mt * kBM + row;
+    valid = tok < p.Mc;
+    nbase = nt * kBN;
+    o = valid ? p.out + static_cast<long long>(__ldg(p.dst + p.tok0 + tok)) * p.d : nullptr;
+  }
+
+  __device__ __forceinline__ void chunk(const Params& p, int c, const uint32_t (&v)[32]) {
+    if (!valid) return;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int col = nbase + c * 32 + q * 4;
+      if (col < p.d)
+        *reinterpret_cast<float4*>(o + col) =
+            make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
+                        __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
+    }
+  }
+
+  __device__ __forceinline__ void end(const Params&) {}
+};
+
+// ------------------------------------------------------------------ dW epilogue
+struct EpiDW {
+  struct Params {
+    float* out;            // dW [V, d]
+    int V, d, accumulate;
+  };
+  float* o;
+  int nbase;
+  bool valid;
+
+  __device__ __forceinline__ void begin(const Params& p, int mt, int nt, int row) {
+    const int v = mt * kBM + row;
+    valid = v < p.V;
+    nbase = nt * kBN;
+    o = valid ? p.out + static_cast<long long>(v) * p.d : nullptr;
+  }
+
+  __device__ __forceinline__ void chunk(const Params& p, int c, const uint32_t (&v)[32]) {
+    if (!valid) return;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int col = nbase + c * 32 + q * 4;
+      if (col < p.d) {
+        float4 r = make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
+                               __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
+        float4* dst = reinterpret_cast<float4*>(o + col);
+        if (p.accumulate) {
+          const float4 old = *dst;
+          r.x += old.x;
+          r.y += old.y;
+          r.z += old.z;
+          r.w += old.w;
+        }
+        *dst = r;
+      }
+    }
+  }
+
+  __device__ __forceinline__ void end(const Params&) {}
+};
+
+template <bool A_MN, bool B_MN, class Epi>
+static cudaError_t run_gemm(const CUtensorMap& mapA, const CUtensorMap& mapB, const GemmGeom& g,
+                            const typename Epi::Params& p, int grid, const DevCtl& ctl,
+                            cudaStream_t st) {
+  auto kern = k_tc_gemm<A_MN, B_MN, Epi>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       kGemmSmemBytes);
+  if (e != cudaSuccess) return e;
+  const int tiles = g.m_tiles * g.n_tiles;
+  if (tiles == 0) return cudaSuccess;
+  kern<<<grid < tiles ? grid : tiles, kGemmThreads, kGemmSmemBytes, st>>>(mapA, mapB, g, p, ctl);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_grad(const CUtensorMap& mapA, const CUtensorMap& mapB, int Mc, int V,
+                            int d, int tok0, const int* y, const float* lse, const float* coef,
+                            const int* rowid, uint16_t* G, long long ldG, int grid,
+                            const DevCtl& ctl, cudaStream_t st) {
+  GemmGeom g{(Mc + kBM - 1) / kBM, (V + kBN - 1) / kBN, (d + kBK - 1) / kBK, 0};
+  EpiGrad::Params p{y, lse, coef, rowid, G, ldG, Mc, V, tok0};
+  return run_gemm<false, false, EpiGrad>(mapA, mapB, g, p, grid, ctl, st);
+}
+
+cudaError_t launch_bwd_dh(const CUtensorMap& mapA, const CUtensorMap& mapB, int Mc, int V, int d,
+                          int tok0, const int* dst, float* dH, int grid, const DevCtl& ctl,
+                          cudaStream_t st) {
+  GemmGeom g{(Mc + kBM - 1) / kBM, (d + kBN - 1) / kBN, (V + kBK - 1) / kBK, 1};
+  EpiRows::Params p{dst, dH, Mc, d, tok0};
+  return run_gemm<false, true, EpiRows>(mapA, mapB, g, p, grid, ctl, st);
+}
+
+cudaError_t launch_bwd_dw(const CUtensorMap& mapA, const CUtensorMap& mapB, int Mc, int V, int d,
+                          float* dW, int accumulate, int grid, const DevCtl& ctl,
+                          cudaStream_t st) {
+  GemmGeom g{(V + kBM - 1) / kBM, (d + kBN - 1) / kBN, (Mc + kBK - 1) / kBK, 1};
+  EpiDW::Params p{dW, V, d, accumulate};
+  return run_gemm<true, true, EpiDW>(mapA, mapB, g, p, grid, ctl, st);
+}
+
+}  // namespace dpo

@@ -1,0 +1,144 @@
+// Exact-fp32 SIMT route for DPO_F32 inputs (small problems; no tensor cores).
+// Same quantities as the bf16 route: per scored position the log-sum-exp over
+// the full vocabulary and the target logit, then dz = coef * (onehot - softmax)
+// and its products with W and H. Each reduction runs in a fixed order.
+#include <cmath>
+
+#include "internal.h"
+
+namespace dpo {
+
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
+}
+
+// z_v = h . W[v] for one vocab row, by one warp (lanes stride over d).
+__device__ __forceinline__ float warp_dot(const float* __restrict__ h,
+                                          const float* __restrict__ w, int d, int lane) {
+  float a = 0.f;
+  for (int k = lane; k < d; k += 32) a = fmaf(__ldg(h + k), __ldg(w + k), a);
+  return warp_sum(a);
+}
+
+// One block per scored position; warp w handles vocab rows w, w + 8, ...
+__global__ void __launch_bounds__(256) k_f32_fwd(const float* __restrict__ H,
+                                                 const float* __restrict__ W, Sched s, int d,
+                                                 int V, float2* __restrict__ part,
+                                                 float* __restrict__ zy) {
+  __shared__ float sm[8], ss[8];
+  const int i = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const float* h = H + static_cast<long long>(s.dst[i]) * d;
+  const int y = s.y[i];
+  float m = -INFINITY, sum = 0.f;
+  for (int v = warp; v < V; v += 8) {
+    const float z = warp_dot(h, W + static_cast<long long>(v) * d, d, lane);
+    if (z > m) {
+      sum = sum * expf(m - z) + 1.f;
+      m = z;
+    } else {
+      sum += expf(z - m);
+    }
+    if (v == y && lane == 0) zy[i] = z;
+  }
+  if (lane == 0) {
+    sm[warp] = m;
+    ss[warp] = sum;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float M = -INFINITY, S = 0.f;
+    for (int w = 0; w < 8; ++w) {
+      if (sm[w] == -INFINITY) continue;            // warp saw no vocab row (V < 8)
+      if (sm[w] > M) {
+        S = S * expf(M - sm[w]) + ss[w];
+        M = sm[w];
+      } else {
+        S += ss[w] * expf(sm[w] - M);
+      }
+    }
+    part[i] = make_float2(M, S);
+  }
+}
+
+cudaError_t launch_f32_fwd(const float* H, const float* W, const Sched& s, int Nc, int d, int V,
+                           float2* part, float* zy, cudaStream_t st) {
+  if (Nc == 0) return cudaSuccess;
+  k_f32_fwd<<<Nc, 256, 0, st>>>(H, W, s, d, V, part, zy);
+  return cudaGetLastError();
+}
+
+// G[i, v] = coef_r * (1[v = y] - exp(z_v - lse)) for positions tok0 + i, i < Mc.
+__global__ void __launch_bounds__(256) k_f32_grad(const float* __restrict__ H,
+                                                  const float* __restrict__ W, Sched s, int tok0,
+                                                  int d, int V, const float* __restrict__ lse,
+                                                  const float* __restrict__ coef,
+                                                  float* __restrict__ G) {
+  const int i = blockIdx.x, gt = tok0 + i;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const float* h = H + static_cast<long long>(s.dst[gt]) * d;
+  const int y = s.y[gt];
+  const float cf = y >= 0 ? coef[s.rowid[gt]] : 0.f;
+  const float l = lse[gt];
+  float* g = G + static_cast<long long>(i) * V;
+  for (int v = warp; v < V; v += 8) {
+    const float z = warp_dot(h, W + static_cast<long long>(v) * d, d, lane);
+    if (lane == 0) g[v] = cf * ((v == y ? 1.f : 0.f) - expf(z - l));
+  }
+}
+
+cudaError_t launch_f32_grad(const float* H, const float* W, const Sched& s, int tok0, int Mc,
+                            int d, int V, const float* lse, const float* coef, float* G,
+                            cudaStream_t st) {
+  if (Mc == 0) return cudaSuccess;
+  k_f32_grad<<<Mc, 256, 0, st>>>(H, W, s, tok0, d, V, lse, coef, G);
+  return cudaGetLastError();
+}
+
+// dH[dst[tok0 + i], k] = sum_v G[i, v] W[v, k]; one block per position.
+__global__ void __launch_bounds__(256) k_f32_dh(const float* __restrict__ G,
+                                                const float* __restrict__ W, Sched s, int tok0,
+                                                int d, int V, float* __restrict__ dH) {
+  const int i = blockIdx.x;
+  const float* g = G + static_cast<long long>(i) * V;
+  float* o = dH + static_cast<long long>(s.dst[tok0 + i]) * d;
+  for (int k = threadIdx.x; k < d; k += blockDim.x) {
+    float a = 0.f;
+    for (int v = 0; v < V; ++v) a = fmaf(__ldg(g + v), __ldg(W + static_cast<long long>(v) * d + k), a);
+    o[k] = a;
+  }
+}
+
+cudaError_t launch_f32_dh(const float* G, const float* W, const Sched& s, int tok0, int Mc, int d,
+                          int V, float* dH, cudaStream_t st) {
+  if (Mc == 0) return cudaSuccess;
+  k_f32_dh<<<Mc, 256, 0, st>>>(G, W, s, tok0, d, V, dH);
+  return cudaGetLastError();
+}
+
+// dW[v, k] (+)= sum_i G[i, v] H[dst[tok0 + i], k]; one block per vocab row.
+__global__ void __launch_bounds__(256) k_f32_dw(const float* __restrict__ G,
+                                                const float* __restrict__ H, Sched s, int tok0,
+                                                int Mc, int d, int V, float* __restrict__ dW,
+                                                int accumulate) {
+  const int v = blockIdx.x;
+  float* o = dW + static_cast<long long>(v) * d;
+  for (int k = threadIdx.x; k < d; k += blockDim.x) {
+    float a = 0.f;
+    for (int i = 0; i < Mc; ++i)
+      a = fmaf(__ldg(G + static_cast<long long>(i) * V + v),
+               __ldg(H + static_cast<long long>(s.dst[tok0 + i]) * d + k), a);
+    o[k] = accumulate ? o[k] + a : a;
+  }
+}
+
+cudaError_t launch_f32_dw(const float* G, const float* H, const Sched& s, int tok0, int Mc, int d,
+                          int V, float* dW, int accumulate, cudaStream_t st) {
+  if (V == 0) return cudaSuccess;
+  k_f32_dw<<<V, 256, 0, st>>>(G, H, s, tok0, Mc, d, V, dW, accumulate);
+  return cudaGetLastError();
+}
+
+}  // namespace dpo

@@ -1,0 +1,93 @@
+// Host-side launchers shared between the library's translation units.
+// Device code lives in the .cu files; this header only declares what the C ABI
+// (api.cu) calls.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "ptx_sm100.cuh"
+#include "tile_config.h"
+
+namespace dpo {
+
+constexpr int kRowChunk = 1024;   // rows uploaded per k_upload_rows launch (kernel parameter)
+
+// Row table slice passed by value to k_upload_rows.
+struct RowChunk {
+  int row0;                       // first row of the slice
+  int n;                          // rows in the slice
+  int R;                          // total rows (row_start has R + 1 entries)
+  int total;                      // Nc, written to row_start[R] by the last slice
+  int rs[kRowChunk];              // packed offset of each row's first scored position
+  int P[kRowChunk];               // prompt length of each row
+};
+
+// Device views of the per-call schedule held in the workspace.
+struct Sched {
+  const int* row_start;   // [R + 1] packed offset of row r's first scored position
+  const int* prompt;      // [R]
+  int* y;                 // [Nc] target token of each scored position (-1 = out of range)
+  int* dst;               // [Nc] flat index r * L + t of each scored position
+  int* rowid;             // [Nc] row of each scored position
+};
+
+cudaError_t launch_upload_rows(const RowChunk& rc, int* row_start, int* prompt,
+                               cudaStream_t st);
+
+// Scored-position tables (y, dst, rowid) and, when Hp != nullptr, the packed
+// bf16 copy of the scored H rows.
+cudaError_t launch_prep(const uint16_t* H, const int* tokens, const Sched& s, int R, int L, int d,
+                        int V, int Nc, uint16_t* Hp, const DevCtl& ctl, cudaStream_t st);
+
+// Forward GEMM with the online log-sum-exp epilogue (bf16, tcgen05).
+//   part[nt * ldp + i] = (max, sum exp(z - max)) of vocab tile nt for packed position i
+//   zy[i] = z at the target column (written by the tile that holds it)
+cudaError_t launch_fwd_lse(const CUtensorMap& mapA, const CUtensorMap& mapB, int Nc, int V,
+                           int d, const int* y, float2* part, int ldp, float* zy, int grid,
+                           const DevCtl& ctl, cudaStream_t st);
+
+// Combine the vocab-tile partials of each position into lse and lp = zy - lse.
+cudaError_t launch_combine(const float2* part, int ldp, int S, const float* zy, const int* y,
+                           int Nc, float* lp, float* lse_out, cudaStream_t st);
+
+// Per-row fp64 sum of lp over the row's scored positions; optional [R, L] token output.
+cudaError_t launch_rowsum(const float* lp, const int* row_start, const int* prompt, int R, int L,
+                          float* seq, float* tok_logp, cudaStream_t st);
+
+// Backward (bf16): G = coef * (onehot - softmax) for packed positions [tok0, tok0 + Mc).
+cudaError_t launch_bwd_grad(const CUtensorMap& mapA, const CUtensorMap& mapB, int Mc, int V,
+                            int d, int tok0, const int* y, const float* lse, const float* coef,
+                            const int* rowid, uint16_t* G, long long ldG, int grid,
+                            const DevCtl& ctl, cudaStream_t st);
+
+// dH rows: out[dst[tok0 + i]] = (G . W)[i]   (A = G K-major, B = W MN-major)
+cudaError_t launch_bwd_dh(const CUtensorMap& mapA, const CUtensorMap& mapB, int Mc, int V, int d,
+                          int tok0, const int* dst, float* dH, int grid, const DevCtl& ctl,
+                          cudaStream_t st);
+
+// dW (+)= G^T . Hp   (A = G MN-major, B = Hp MN-major)
+cudaError_t launch_bwd_dw(const CUtensorMap& mapA, const CUtensorMap& mapB, int Mc, int V, int d,
+                          float* dW, int accumulate, int grid, const DevCtl& ctl,
+                          cudaStream_t st);
+
+// Loss kernel (fp64 inside).
+cudaError_t launch_loss(int B, int layout, const float* pol, const float* ref, double beta,
+                        double grad_scale, float* loss, float* accuracy, float* margins,
+                        float* chosen_rewards, float* rejected_rewards, float* weights,
+                        float* row_coef, cudaStream_t st);
+
+// fp32 SIMT path.
+cudaError_t launch_f32_fwd(const float* H, const float* W, const Sched& s, int Nc, int d, int V,
+                           float2* part, float* zy, cudaStream_t st);
+cudaError_t launch_f32_grad(const float* H, const float* W, const Sched& s, int tok0, int Mc,
+                            int d, int V, const float* lse, const float* coef, float* G,
+                            cudaStream_t st);
+cudaError_t launch_f32_dh(const float* G, const float* W, const Sched& s, int tok0, int Mc, int d,
+                          int V, float* dH, cudaStream_t st);
+cudaError_t launch_f32_dw(const float* G, const float* H, const Sched& s, int tok0, int Mc, int d,
+                          int V, float* dW, int accumulate, cudaStream_t st);
+
+}  // namespace dpo

@@ -1,0 +1,259 @@
+// Persistent, warp-specialised bf16 GEMM on the 5th-generation tensor cores
+// (tcgen05.mma, cta_group::1) with a pluggable per-row epilogue.
+//
+//   D[M x N] = A[M x K] . B[N x K]^T     (fp32 accumulation in tensor memory)
+//
+// A and B are fed from global memory by TMA into a STAGES-deep ring of
+// 128-byte-swizzled shared-memory tiles. Each operand can be K-major (rows of K
+// contiguous) or MN-major (rows of M or N contiguous, i.e. the transposed
+// storage); the shared-memory descriptor and the TMA boxes follow.
+//
+// Roles (192 threads, one CTA per SM, persistent over a static tile schedule):
+//   warp 0     one thread issues the TMA loads,
+//   warp 1     allocates 512 TMEM columns; one thread issues the MMAs,
+//   warps 2-5  epilogue: each thread owns one accumulator row (TMEM lane) and
+//              reads its 256 fp32 columns in 8 chunks of 32 (tcgen05.ld).
+// The accumulator is double-buffered (2 x 256 columns) so the epilogue of tile
+// i overlaps the main loop of tile i+1.
+#pragma once
+
+#include "ptx_sm100.cuh"
+#include "tile_config.h"
+
+namespace dpo {
+
+constexpr int kStages = 4;
+constexpr int kABytes = kBM * kBK * 2;   // 16 KiB
+constexpr int kBBytes = kBN * kBK * 2;   // 32 KiB
+constexpr int kStageBytes = kABytes + kBBytes;
+constexpr int kGemmThreads = 192;
+constexpr int kTmemCols = 512;
+constexpr int kGemmSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+
+// Tile schedule: linear tile index -> (m tile, n tile).
+//   order 0: m fastest (all M tiles of one N tile run together: B tile shared via L2)
+//   order 1: n fastest (all N tiles of one M tile run together: A tile shared via L2)
+struct GemmGeom {
+  int m_tiles, n_tiles, k_blocks;
+  int order;
+};
+
+__device__ __forceinline__ void tile_coords(const GemmGeom& g, int tile, int& mt, int& nt) {
+  if (g.order == 0) {
+    mt = tile % g.m_tiles;
+    nt = tile / g.m_tiles;
+  } else {
+    mt = tile / g.n_tiles;
+    nt = tile % g.n_tiles;
+  }
+}
+
+// Epilogue interface (one object per epilogue thread, per tile):
+//   __device__ void begin(const Params&, int mt, int nt, int row);
+//   __device__ void chunk(const Params&, int c, const uint32_t (&v)[32]);   // columns c*32..+31
+//   __device__ void end(const Params&);
+template <bool A_MN, bool B_MN, class Epi>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    k_tc_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+              GemmGeom g, typename Epi::Params ep, DevCtl ctl) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem;                                  // kStages x 16 KiB
+  uint8_t* sB = smem + kStages * kABytes;              // kStages x 32 KiB
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
+  // bars[0..S)   full      (TMA -> MMA)
+  // bars[S..2S)  empty     (MMA -> TMA)
+  // bars[2S..2S+2) acc_full  (MMA -> epilogue)
+  // bars[2S+2..2S+4) acc_empty (epilogue -> MMA)
+  // bars[2S+4]   drain     (MMA teardown)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 5);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t full0 = smem_u32(bars);
+  const uint32_t empty0 = smem_u32(bars + kStages);
+  const uint32_t accf0 = smem_u32(bars + 2 * kStages);
+  const uint32_t acce0 = smem_u32(bars + 2 * kStages + 2);
+  const uint32_t drain = smem_u32(bars + 2 * kStages + 4);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(accf0 + 8 * a, 1);
+      mbar_init(acce0 + 8 * a, 4 * 32);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int n_tiles_total = g.m_tiles * g.n_tiles;
+  // Producer bookkeeping kept for the teardown: which stages have a load issued
+  // and the parity of the `full` phase that load completes.
+  uint32_t issued_mask = 0, issued_par = 0;
+
+  if (warp == 0 && lane == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < n_tiles_total && ok; tile += gridDim.x) {
+      int mt, nt;
+      tile_coords(g, tile, mt, nt);
+      for (int kb = 0; kb < g.k_blocks; ++kb) {
+        if (!mbar_wait(empty0 + 8 * stage, phase ^ 1, ctl, abort_flag)) {
+          ok = false;
+          break;
+        }
+        const uint32_t fb = full0 + 8 * stage;
+        mbar_arrive_expect_tx(fb, kStageBytes);
+        const uint32_t a_dst = smem_u32(sA + stage * kABytes);
+        const uint32_t b_dst = smem_u32(sB + stage * kBBytes);
+        if (!A_MN) {
+          tma_load_2d(a_dst, &tmA, fb, kb * kBK, mt * kBM);
+        } else {
+#pragma unroll
+          for (int j = 0; j < kBM / 64; ++j)
+            tma_load_2d(a_dst + j * 8192, &tmA, fb, mt * kBM + j * 64, kb * kBK);
+        }
+        if (!B_MN) {
+          tma_load_2d(b_dst, &tmB, fb, kb * kBK, nt * kBN);
+        } else {
+#pragma unroll
+          for (int j = 0; j < kBN / 64; ++j)
+            tma_load_2d(b_dst + j * 8192, &tmB, fb, nt * kBN + j * 64, kb * kBK);
+        }
+        issued_mask |= 1u << stage;
+        issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+        if (++stage == kStages) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+    }
+    if (!ok) {
+      record_status(ctl, kStatusTimeout);
+      *abort_flag = 1;
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ---------------------------------------------------------------- MMA issuer
+    constexpr uint32_t idesc = idesc_bf16_f32(kBM, kBN, A_MN, B_MN);
+    int stage = 0;
+    uint32_t phase = 0;
+    int local = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < n_tiles_total && ok; tile += gridDim.x, ++local) {
+      const int acc = local & 1;
+      const uint32_t acc_phase = (local >> 1) & 1;
+      if (!mbar_wait(acce0 + 8 * acc, acc_phase ^ 1, ctl, abort_flag)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + acc * kBN;
+      for (int kb = 0; kb < g.k_blocks; ++kb) {
+        if (!mbar_wait(full0 + 8 * stage, phase, ctl, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a0 = smem_u32(sA + stage * kABytes);
+        const uint32_t b0 = smem_u32(sB + stage * kBBytes);
+#pragma unroll
+        for (int k = 0; k < kBK / 16; ++k) {
+          // K-major: the 16-wide K slice sits 32 bytes further along the swizzled row.
+          // MN-major: it is the next 16 rows of K, 16 * 128 bytes further.
+          const uint64_t ad = A_MN ? sw128_desc(a0 + k * 2048, 8192, 1024)
+                                   : sw128_desc(a0 + k * 32, 16, 1024);
+          const uint64_t bd = B_MN ? sw128_desc(b0 + k * 2048, 8192, 1024)
+                                   : sw128_desc(b0 + k * 32, 16, 1024);
+          tc_mma_f16(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
+        }
+        tc_commit(empty0 + 8 * stage);   // frees this stage once its MMAs are done
+        if (++stage == kStages) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+      if (!ok) break;
+      tc_commit(accf0 + 8 * acc);        // accumulator ready for the epilogue
+    }
+    if (!ok) {
+      record_status(ctl, kStatusTimeout);
+      *abort_flag = 1;
+    }
+    // Drain: wait (bounded) until every MMA issued by this thread has completed,
+    // so TMEM is not freed under an MMA in flight.
+    tc_commit(drain);
+    DevCtl c2 = ctl;
+    volatile int never = 0;
+    if (!mbar_wait(drain, 0, c2, &never)) record_status(ctl, kStatusTimeout);
+  } else if (warp >= 2) {
+    // ---------------------------------------------------------------- epilogue
+    const int lg = warp & 3;                 // TMEM lane group this warp may access
+    const int row = lg * 32 + lane;
+    const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(lg * 32) << 16);
+    int local = 0;
+    for (int tile = blockIdx.x; tile < n_tiles_total; tile += gridDim.x, ++local) {
+      const int acc = local & 1;
+      const uint32_t acc_phase = (local >> 1) & 1;
+      if (!mbar_wait(accf0 + 8 * acc, acc_phase, ctl, abort_flag)) {
+        record_status(ctl, kStatusTimeout);
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      int mt, nt;
+      tile_coords(g, tile, mt, nt);
+      Epi epi;
+      epi.begin(ep, mt, nt, row);
+#pragma unroll 1
+      for (int c = 0; c < kBN / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(lane_addr + acc * kBN + c * 32, v);
+        tmem_wait_ld();
+        epi.chunk(ep, c, v);
+      }
+      tc_fence_before();
+      mbar_arrive(acce0 + 8 * acc);
+      epi.end(ep);
+    }
+  }
+
+  // ---------------------------------------------------------------- teardown
+  __syncthreads();
+  if (warp == 0 && lane == 0 && *abort_flag) {
+    // After an abort, loads may still be in flight into shared memory: wait
+    // (bounded) for the phase each stage's last load completes before the CTA
+    // exits. A phase that already completed returns at once.
+    volatile int never = 0;
+    DevCtl c2 = ctl;
+    c2.budget_ns = ctl.budget_ns / 4 + 1000000ull;
+    for (int s = 0; s < kStages; ++s)
+      if (issued_mask & (1u << s))
+        (void)mbar_wait(full0 + 8 * s, (issued_par >> s) & 1u, c2, &never);
+  }
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+}  // namespace dpo

@@ -1,0 +1,188 @@
+"""ctypes binding of libdpo (include/dpo.h): argument marshalling only.
+
+Every step of the DPO head path runs in the CUDA library; this module turns
+Python arguments into the C ABI's plain pointers and sizes. Device buffers may
+be given as torch tensors (their data_ptr() is passed) or as integer device
+addresses; host row-length arrays as numpy int32 arrays. The names follow the C
+entry points without the `dpo_` prefix.
+
+The module refuses to run without the compiled library: there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "lib", "libdpo.so")
+
+# dpo_status
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_BAD_TARGET, ERR_WORKSPACE = range(7)
+# dpo_dtype
+BF16, F32, F16 = 0, 1, 2
+# dpo_layout
+PAIRS_HALVES, PAIRS_ADJACENT = 0, 1
+
+LAYOUTS = {"halves": PAIRS_HALVES, "adjacent": PAIRS_ADJACENT}
+DTYPES = {"bf16": BF16, "f32": F32, "f16": F16}
+
+
+class DpoError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+
+
+class Batch(ctypes.Structure):
+    _fields_ = [
+        ("R", ctypes.c_int32), ("L", ctypes.c_int32), ("d", ctypes.c_int32), ("V", ctypes.c_int32),
+        ("dtype", ctypes.c_int32),
+        ("H", ctypes.c_void_p), ("W", ctypes.c_void_p), ("tokens", ctypes.c_void_p),
+        ("prompt_len", ctypes.c_void_p), ("completion_len", ctypes.c_void_p),
+    ]
+
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libdpo.so (built in-tree by preference_alignment_b200.build)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"libdpo.so is not built ({path}); run "
+                           "`python -m preference_alignment_b200.build`")
+    lib = ctypes.CDLL(path)
+    vp, sz, i32, u32, f32 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32, ctypes.c_uint32, ctypes.c_float
+    bp = ctypes.POINTER(Batch)
+    szp = ctypes.POINTER(ctypes.c_size_t)
+    lib.dpo_workspace_size.argtypes = [bp, szp, szp, szp]
+    lib.dpo_seq_logprobs.argtypes = [bp, ctypes.c_int, vp, vp, vp, vp, sz, vp]
+    lib.dpo_loss.argtypes = [i32, i32, vp, vp, f32, f32, vp, vp, vp, vp, vp, vp, vp, vp]
+    lib.dpo_backward.argtypes = [bp, vp, vp, vp, vp, ctypes.c_int, vp, sz, vp]
+    lib.dpo_check.argtypes = [vp]
+    lib.dpo_set_wait_budget_ms.argtypes = [u32]
+    lib.dpo_set_wait_budget_ms.restype = u32
+    lib.dpo_status_string.argtypes = [ctypes.c_int]
+    lib.dpo_status_string.restype = ctypes.c_char_p
+    lib.dpo_version.restype = i32
+    for name in ("dpo_workspace_size", "dpo_seq_logprobs", "dpo_loss", "dpo_backward", "dpo_check"):
+        getattr(lib, name).restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def _ptr(x) -> Optional[int]:
+    """Device/host address of a torch tensor, numpy array or raw integer; None -> NULL."""
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    if hasattr(x, "data_ptr"):
+        return x.data_ptr()
+    if isinstance(x, np.ndarray):
+        return x.ctypes.data
+    raise TypeError(f"cannot take the address of {type(x)}")
+
+
+def _stream(s) -> Optional[int]:
+    if s is None:
+        try:
+            import torch
+            if torch.cuda.is_available():
+                return torch.cuda.current_stream().cuda_stream
+        except Exception:
+            pass
+        return None
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream
+
+
+def _check(status: int, where: str):
+    if status != OK:
+        raise DpoError(status, where)
+
+
+def status_string(status: int) -> str:
+    return load().dpo_status_string(int(status)).decode()
+
+
+def version() -> int:
+    return load().dpo_version()
+
+
+def set_wait_budget_ms(ms: int) -> int:
+    return load().dpo_set_wait_budget_ms(int(ms))
+
+
+class BatchArgs:
+    """A dpo_batch plus the Python objects its pointers refer to (kept alive)."""
+
+    def __init__(self, H, W, tokens, prompt_len, completion_len, R=None, L=None, d=None, V=None,
+                 dtype="bf16"):
+        self.prompt_len = np.ascontiguousarray(prompt_len, dtype=np.int32)
+        self.completion_len = np.ascontiguousarray(completion_len, dtype=np.int32)
+        shapeH = tuple(H.shape) if hasattr(H, "shape") else None
+        shapeW = tuple(W.shape) if hasattr(W, "shape") else None
+        R = R if R is not None else shapeH[0]
+        L = L if L is not None else shapeH[1]
+        d = d if d is not None else shapeH[2]
+        V = V if V is not None else shapeW[0]
+        self.keep = (H, W, tokens)
+        self.c = Batch(int(R), int(L), int(d), int(V), DTYPES.get(dtype, dtype) if isinstance(dtype, str) else int(dtype),
+                       _ptr(H), _ptr(W), _ptr(tokens), self.prompt_len.ctypes.data,
+                       self.completion_len.ctypes.data)
+
+    @property
+    def n_scored(self) -> int:
+        return int(self.completion_len.sum())
+
+
+def workspace_size(batch: BatchArgs):
+    """(fwd_bytes, bwd_bytes, bwd_min_bytes) for this batch."""
+    f, b, m = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    _check(load().dpo_workspace_size(ctypes.byref(batch.c), ctypes.byref(f), ctypes.byref(b),
+                                     ctypes.byref(m)), "dpo_workspace_size")
+    return f.value, b.value, m.value
+
+
+def _nbytes(ws, ws_bytes):
+    if ws_bytes is not None:
+        return int(ws_bytes)
+    if hasattr(ws, "numel"):
+        return ws.numel() * ws.element_size()
+    raise ValueError("ws_bytes is required for a raw workspace address")
+
+
+def seq_logprobs(batch: BatchArgs, want_grad: bool, seq_logp, tok_logp, lse_state, ws,
+                 ws_bytes=None, stream=None):
+    _check(load().dpo_seq_logprobs(ctypes.byref(batch.c), 1 if want_grad else 0, _ptr(seq_logp),
+                                   _ptr(tok_logp), _ptr(lse_state), _ptr(ws), _nbytes(ws, ws_bytes),
+                                   _stream(stream)), "dpo_seq_logprobs")
+
+
+def loss(B: int, layout, pol, ref, beta: float, grad_scale: float, loss_out, accuracy=None,
+         margins=None, chosen_rewards=None, rejected_rewards=None, weights=None, row_coef=None,
+         stream=None):
+    lay = LAYOUTS[layout] if isinstance(layout, str) else int(layout)
+    _check(load().dpo_loss(int(B), lay, _ptr(pol), _ptr(ref), float(beta), float(grad_scale),
+                           _ptr(loss_out), _ptr(accuracy), _ptr(margins), _ptr(chosen_rewards),
+                           _ptr(rejected_rewards), _ptr(weights), _ptr(row_coef), _stream(stream)),
+           "dpo_loss")
+
+
+def backward(batch: BatchArgs, lse_state, row_coef, dH, dW, accumulate_dW: bool, ws,
+             ws_bytes=None, stream=None):
+    _check(load().dpo_backward(ctypes.byref(batch.c), _ptr(lse_state), _ptr(row_coef), _ptr(dH),
+                               _ptr(dW), 1 if accumulate_dW else 0, _ptr(ws),
+                               _nbytes(ws, ws_bytes), _stream(stream)), "dpo_backward")
+
+
+def check(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device status word."""
+    return load().dpo_check(_stream(stream))
