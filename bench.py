@@ -1,0 +1,446 @@
+"""Benchmark of the fused DPO head step on B200 through libdpo's C ABI.
+
+One step = policy dpo_seq_logprobs(want_grad=1) + reference dpo_seq_logprobs
++ dpo_loss + dpo_backward, on the Llama-3.1-8B head shape (8 rows = 4
+chosen/rejected pairs, L = 2048, d = 4096, V = 128,256, bf16), synthetic seeded
+inputs. Under torchrun each rank runs its own pairs (data parallel, weak
+scaling) with the same weights; the step ends with an NCCL all-reduce of dW and
+of the loss, the exchange a data-parallel optimiser step needs.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Rank 0 prints one JSON line. The value is scored completion tokens per second
+over all ranks (max time over ranks, CUDA events, inputs resident in HBM).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from preference_alignment_b200 import workloads as WL  # noqa: E402
+
+METRIC = "DPO fwd+bwd tokens/s on 1 B200; % of bf16 dense tensor-core peak"
+UNIT = "tokens/s"
+WORKLOAD = "llama8b"
+CONFIG_TEXT = ("Llama-3.1-8B head shape: 4 pairs -> 8 rows, seq 2048, prompt U{256..1024}, "
+               "completion to >=95% fill, d=4096, V=128256, bf16; policy fwd+bwd, reference fwd")
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ------------------------------------------------------------------ helpers
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return PEAKS_FALLBACK, "fallback"
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def rank_workload(name, rank):
+    """The named workload with this rank's own batch (same weights on every rank)."""
+    w = WL.make_config(name)
+    if rank == 0:
+        return w
+    idx, R, L, d, V, dtype, layout, ref_std, rule, _ = WL.CONFIGS[name]
+    rng = np.random.Generator(np.random.PCG64([w.seed, rank]))
+    P, C = rule(rng, R, L)
+    w.prompt_len = P.astype(np.int32)
+    w.completion_len = C.astype(np.int32)
+    w.tokens = rng.integers(0, V, size=(R, L), dtype=np.int64).astype(np.int32)
+    w.H = WL.bf16_bits_from_f32(rng.standard_normal(size=(R, L, d), dtype=np.float32))
+    return w
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+                except ValueError:
+                    continue
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, fl in rows for i, v in enumerate(fl) if v.lower() == "active"})
+        sm = [r[0] for r in rows]
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": max(r[1] for r in rows),
+                "samples": len(rows), "reasons": reasons}
+
+
+# ------------------------------------------------------------------ oracle sample (host cores)
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+class OracleSample:
+    """The CPU fp64 oracle on a bounded sample of the workload: one pair (a chosen
+    and a rejected row) with its completions cut to `per_row` tokens each, full
+    d and V: policy forward, reference forward, loss and backward to dH and dW,
+    the same work per token as the GPU step."""
+
+    def __init__(self, w, per_row):
+        from oracle import dpo_oracle as O
+        self.O = O
+        self.w = w
+        B = w.R // 2
+        rows = [0, B] if w.layout == "halves" else [0, 1]
+        self.H = WL.widen(w.H[rows], w.dtype)
+        self.tokens = w.tokens[rows]
+        self.P = w.prompt_len[rows].copy()
+        self.C = np.minimum(w.completion_len[rows], per_row).astype(np.int32)
+        self.W = WL.widen(w.W, w.dtype)
+        self.Wr = WL.widen(w.W_ref, w.dtype) if w.W_ref is not None else None
+        self.n_tokens = int(self.C.sum())
+
+    def step(self):
+        O = self.O
+        pol = O.seq_logprobs(self.H, self.W, self.tokens, self.P, self.C)["seq_logp"]
+        if self.Wr is None:
+            return
+        ref = O.seq_logprobs(self.H, self.Wr, self.tokens, self.P, self.C)["seq_logp"]
+        lo = O.dpo_loss(pol, ref, self.w.beta, "halves")
+        O.backward(self.H, self.W, self.tokens, self.P, self.C, lo["row_coef"])
+
+
+def run_reference(args):
+    """The oracle as the reference arm: K timed steps of a bounded sample on host cores."""
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    w = WL.make_config(args.workload)
+    s = OracleSample(w, per_row=args.ref_tokens_per_row)
+    for _ in range(args.warmup):
+        s.step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        s.step()
+    dt = time.perf_counter() - t0
+    value = s.n_tokens * args.steps / dt
+    cores = blas_threads()
+    sample = (f"oracle fp64 (numpy/OpenBLAS) on one pair of the {args.workload} workload, "
+              f"completions cut to {args.ref_tokens_per_row} tokens per row ({s.n_tokens} tokens/step), "
+              f"full d and V; policy fwd + reference fwd + loss + backward")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": args.workload, "text": CONFIG_TEXT},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def cpu_baseline(w, per_row):
+    s = OracleSample(w, per_row=per_row)
+    s.step()                                   # warm caches / page in the widened weights
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        s.step()
+        n += 1
+        if time.perf_counter() - t0 > 8.0 or n >= 3:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": s.n_tokens * n / dt, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": (f"oracle fp64 on one pair of the {w.name} workload with completions cut to "
+                       f"{per_row} tokens per row ({s.n_tokens} tokens), full d={w.d} and V={w.V}; "
+                       f"policy fwd + reference fwd + loss + backward; {n} timed repetitions")}
+
+
+# ------------------------------------------------------------------ GPU arm
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from preference_alignment_b200 import libdpo
+
+    ws_n, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws_n > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    libdpo.load()
+
+    w = rank_workload(args.workload, rank)
+    B = w.R // 2
+
+    def dev_bf16(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    H = dev_bf16(w.H)
+    W = dev_bf16(w.W)
+    fwd_only = w.W_ref is None               # offline reference scoring: forward only
+    Wr = dev_bf16(w.W_ref) if not fwd_only else None
+    tokens = torch.from_numpy(w.tokens).to(dev)
+    bp = libdpo.BatchArgs(H, W, tokens, w.prompt_len, w.completion_len, dtype="bf16")
+    br = libdpo.BatchArgs(H, Wr, tokens, w.prompt_len, w.completion_len, dtype="bf16") if not fwd_only else None
+    fwd_b, bwd_b, _ = libdpo.workspace_size(bp)
+    ws = torch.empty(fwd_b if fwd_only else max(fwd_b, bwd_b), dtype=torch.uint8, device=dev)
+    Nc = w.n_scored
+    pol = torch.empty(w.R, device=dev)
+    ref = torch.empty(w.R, device=dev)
+    lse = torch.empty(Nc, device=dev)
+    dH = torch.empty(w.R, w.L, w.d, device=dev) if not fwd_only else None
+    dW = torch.empty(w.V, w.d, device=dev) if not fwd_only else None
+    outs = {k: torch.empty(n, device=dev) for k, n in
+            [("loss", 1), ("accuracy", 1), ("margins", B), ("cr", B), ("rr", B), ("w", B),
+             ("coef", 2 * B)]}
+    stream = torch.cuda.current_stream(dev)
+    sp = stream.cuda_stream
+    grad_scale = 1.0 / ws_n                  # loss is the mean over the global batch
+
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+
+    def step(timed=None):
+        if fwd_only:
+            if timed is not None:
+                ev[0].record(stream)
+            libdpo.seq_logprobs(bp, False, pol, None, None, ws, stream=sp)
+            if timed is not None:
+                ev[1].record(stream)
+                torch.cuda.synchronize(dev)
+                timed.append([ev[0].elapsed_time(ev[1])] * 2 + [0.0, 0.0])
+            return
+        if timed is not None:
+            ev[0].record(stream)
+        libdpo.seq_logprobs(bp, True, pol, None, lse, ws, stream=sp)
+        if timed is not None:
+            ev[1].record(stream)
+        libdpo.seq_logprobs(br, False, ref, None, None, ws, stream=sp)
+        if timed is not None:
+            ev[2].record(stream)
+        libdpo.loss(B, w.layout, pol, ref, w.beta, grad_scale, outs["loss"], outs["accuracy"],
+                    outs["margins"], outs["cr"], outs["rr"], outs["w"], outs["coef"], stream=sp)
+        if timed is not None:
+            ev[3].record(stream)
+        libdpo.backward(bp, lse, outs["coef"], dH, dW, False, ws, stream=sp)
+        if timed is not None:
+            ev[4].record(stream)
+            torch.cuda.synchronize(dev)
+            timed.append([ev[i].elapsed_time(ev[i + 1]) for i in range(4)])
+        if ws_n > 1:
+            dist.all_reduce(dW)
+            dist.all_reduce(outs["loss"])
+            outs["loss"].mul_(1.0 / ws_n)
+
+    # launches of our kernels per step: upload + prep + GEMM + combine + rowsum per forward,
+    # one loss kernel, upload + prep + 3 GEMMs for the backward (one token chunk: the
+    # workspace holds all Nc rows of dz)
+    uploads = math.ceil(w.R / 1024)
+    fwd_launches = uploads + 4
+    launches_per_step = (fwd_launches if fwd_only else 2 * fwd_launches + 1 + uploads + 4)
+
+    for _ in range(args.warmup):
+        step()
+    st = libdpo.check(sp)
+    if st != libdpo.OK:
+        raise RuntimeError(f"device status after warm-up: {libdpo.status_string(st)}")
+
+    # per-call breakdown (separate short pass with a sync after each step)
+    breakdown = []
+    for _ in range(min(5, args.steps)):
+        step(timed=breakdown)
+    bd = np.median(np.array(breakdown), axis=0)
+
+    clocks = ClockSampler(local)
+    if ws_n > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    time.sleep(0.3)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for _ in range(args.steps):
+        step()
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    if ws_n > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    ms = t_start.elapsed_time(t_end)
+    st = libdpo.check(sp)
+    if st != libdpo.OK:
+        raise RuntimeError(f"device status after timing: {libdpo.status_string(st)}")
+
+    # ------------------------------------------------------------ end to end (host buffers)
+    H_host = torch.from_numpy(np.ascontiguousarray(w.H).view(np.int16)).view(torch.bfloat16).pin_memory()
+    tok_host = torch.from_numpy(w.tokens).pin_memory()
+    res_host = torch.empty(max(2 + 3 * B, w.R), dtype=torch.float32).pin_memory()
+    e2e_steps = max(3, min(args.steps, 20))
+    if ws_n > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        H.copy_(H_host, non_blocking=True)
+        tokens.copy_(tok_host, non_blocking=True)
+        step()
+        if fwd_only:
+            res_dev = pol
+        else:
+            res_dev = torch.cat([outs["loss"], outs["accuracy"], outs["margins"], outs["cr"], outs["rr"]])
+        res_host[:res_dev.numel()].copy_(res_dev, non_blocking=True)
+        stream.synchronize()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1)
+    h2d = H_host.numel() * 2 + tok_host.numel() * 4
+    d2h = (w.R if fwd_only else 2 + 3 * B) * 4
+
+    # ------------------------------------------------------------ aggregate over ranks
+    t = torch.tensor([ms, e2e_ms, float(Nc)], device=dev, dtype=torch.float64)
+    if ws_n > 1:
+        tmax = t.clone()
+        dist.all_reduce(tmax, op=dist.ReduceOp.MAX)
+        tsum = t.clone()
+        dist.all_reduce(tsum, op=dist.ReduceOp.SUM)
+        ms, e2e_ms = float(tmax[0]), float(tmax[1])
+        total_nc = float(tsum[2])
+    else:
+        total_nc = float(Nc)
+
+    peaks, peak_src = load_peaks()
+    value = total_nc * args.steps / (ms / 1e3)
+    e2e_value = total_nc * e2e_steps / (e2e_ms / 1e3)
+    ms_step = ms / args.steps
+    gemm_flop = 2.0 * Nc * w.d * w.V                      # one LM-head GEMM over scored tokens
+    alg_flop = (1 if fwd_only else 4) * gemm_flop          # policy fwd, ref fwd, dH, dW
+    exe_flop = (1 if fwd_only else 5) * gemm_flop          # + backward logit recompute
+    sustained = float(peaks.get("bf16_tflops_sustained", PEAKS_FALLBACK["bf16_tflops_sustained"]))
+    # dominant kernel: the forward LSE GEMM (two launches per step), timed by the events
+    # around the reference dpo_seq_logprobs call (the call also runs the small prep,
+    # combine and row-sum kernels, so the figure is a slight underestimate)
+    fwd_ms = float(bd[1])
+    fwd_tflops = gemm_flop / (fwd_ms / 1e3) / 1e12
+    line = None
+    if rank == 0:
+        cpu = None
+        if ws_n == 1 and not args.no_cpu_baseline:
+            cpu = cpu_baseline(w, per_row=args.cpu_tokens_per_row)
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws_n, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded; random-init LM-head weights of the Llama-3.1-8B head shape)",
+            "config": {"workload": args.workload, "text": CONFIG_TEXT, "rows_per_gpu": w.R,
+                       "pairs_per_gpu": B, "seq_len": w.L, "d": w.d, "V": w.V,
+                       "scored_tokens_per_gpu": Nc, "global_batch_pairs": B * ws_n,
+                       "parallelism": f"dp{ws_n}",
+                       "l2": "inputs larger than L2 (W and W_ref are 1.05 GB each; no flush)"},
+            "pct_of_peak": {"algorithmic": alg_flop * args.steps / (ms / 1e3) / 1e12 / sustained,
+                            "executed": exe_flop * args.steps / (ms / 1e3) / 1e12 / sustained,
+                            "peak_tflops": sustained, "peak": f"bf16 sustained, {peak_src}",
+                            "flop_per_step_algorithmic": alg_flop,
+                            "flop_per_step_executed": exe_flop},
+            "batch_tokens_per_s": w.R * w.L * ws_n * args.steps / (ms / 1e3),
+            "breakdown_ms": {"policy_fwd": float(bd[0]), "ref_fwd": float(bd[1]),
+                             "loss": float(bd[2]), "backward": float(bd[3])},
+            "roofline": {"kernel": "k_tc_gemm<EpiLSE> (forward LM-head GEMM + online LSE)",
+                         "bound": "tensor", "achieved": fwd_tflops, "peak": sustained,
+                         "unit": "TFLOP/s", "frac": fwd_tflops / sustained,
+                         "traffic": None,
+                         "algorithmic_per_launch": f"2*Nc*d*V = {gemm_flop:.4g} FLOP",
+                         "peak_kind": f"bf16_tflops_sustained ({peak_src})"},
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clk,
+            "cpu_baseline": cpu,
+            "peak_device_bytes": torch.cuda.max_memory_allocated(dev),
+            "logits_fp32_bytes_avoided": 4 * Nc * w.V,
+        }
+        print(json.dumps(line), flush=True)
+    if ws_n > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=WORKLOAD, choices=sorted(WL.CONFIGS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-tokens-per-row", type=int, default=64)
+    ap.add_argument("--ref-tokens-per-row", type=int, default=4)
+    args = ap.parse_args(argv)
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())
