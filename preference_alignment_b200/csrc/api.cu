@@ -250,8 +250,8 @@ dpo_status dpo_seq_logprobs(const dpo_batch* batch, int want_grad, float* seq_lo
   if (p.Nc > 0) {
     if (p.dtype == DPO_BF16) {
       CUtensorMap mA, mB;
-      if (!make_map(&mA, w + p.off_hp, p.d, p.Nc, 2ull * p.d, kBK, kBM) ||
-          !make_map(&mB, batch->W, p.d, p.V, 2ull * p.d, kBK, kBN))
+      if (!make_map(&mA, w + p.off_hp, p.d, p.Nc, 2ull * p.d, kBK, kBoxRows) ||
+          !make_map(&mB, batch->W, p.d, p.V, 2ull * p.d, kBK, kBoxRows))
         return DPO_ERR_CUDA;
       if (launch_fwd_lse(mA, mB, p.Nc, p.V, p.d, sc.y, part, p.ldp, zy, di.sms, ctl, st) !=
           cudaSuccess)
@@ -324,12 +324,12 @@ dpo_status dpo_backward(const dpo_batch* batch, const float* lse_state, const fl
       uint16_t* G = reinterpret_cast<uint16_t*>(w + p.off_G);
       const uint16_t* hp0 = Hp + static_cast<size_t>(tok0) * p.d;
       CUtensorMap mHk, mWk, mGk, mWmn, mGmn, mHmn;
-      if (!make_map(&mHk, hp0, p.d, mc, 2ull * p.d, kBK, kBM) ||
-          !make_map(&mWk, batch->W, p.d, p.V, 2ull * p.d, kBK, kBN) ||
-          !make_map(&mGk, G, p.V, mc, 2ull * p.ldG, kBK, kBM) ||
-          !make_map(&mWmn, batch->W, p.d, p.V, 2ull * p.d, 64, kBK) ||
-          !make_map(&mGmn, G, p.V, mc, 2ull * p.ldG, 64, kBK) ||
-          !make_map(&mHmn, hp0, p.d, mc, 2ull * p.d, 64, kBK))
+      if (!make_map(&mHk, hp0, p.d, mc, 2ull * p.d, kBK, kBoxRows) ||
+          !make_map(&mWk, batch->W, p.d, p.V, 2ull * p.d, kBK, kBoxRows) ||
+          !make_map(&mGk, G, p.V, mc, 2ull * p.ldG, kBK, kBoxRows) ||
+          !make_map(&mWmn, batch->W, p.d, p.V, 2ull * p.d, kBoxMN, kBK) ||
+          !make_map(&mGmn, G, p.V, mc, 2ull * p.ldG, kBoxMN, kBK) ||
+          !make_map(&mHmn, hp0, p.d, mc, 2ull * p.d, kBoxMN, kBK))
         return DPO_ERR_CUDA;
       if (launch_bwd_grad(mHk, mWk, mc, p.V, p.d, tok0, sc.y, lse_state, row_coef, sc.rowid, G,
                           p.ldG, di.sms, ctl, st) != cudaSuccess)

@@ -16,7 +16,7 @@
 #include <cmath>
 
 #include "internal.h"
-#include "tc_gemm.cuh"
+#include "gemm_launch.cuh"
 
 namespace dpo {
 
@@ -38,8 +38,8 @@ struct EpiGrad {
   float nl2, cf;
   uint16_t* out;
 
-  __device__ __forceinline__ void begin(const Params& p, int mt, int nt, int row) {
-    const int tok = mt * kBM + row;
+  __device__ __forceinline__ void begin(const Params& p, int m_row, int nt) {
+    const int tok = m_row;
     valid = tok < p.Mc;
     vbase = nt * kBN;
     yl = -1;
@@ -92,8 +92,8 @@ struct EpiRows {
   int nbase;
   bool valid;
 
-  __device__ __forceinline__ void begin(const Params& p, int mt, int nt, int row) {
-    const int tok = mt * kBM + row;
+  __device__ __forceinline__ void begin(const Params& p, int m_row, int nt) {
+    const int tok = m_row;
     valid = tok < p.Mc;
     nbase = nt * kBN;
     o = valid ? p.out + static_cast<long long>(__ldg(p.dst + p.tok0 + tok)) * p.d : nullptr;
@@ -124,8 +124,8 @@ struct EpiDW {
   int nbase;
   bool valid;
 
-  __device__ __forceinline__ void begin(const Params& p, int mt, int nt, int row) {
-    const int v = mt * kBM + row;
+  __device__ __forceinline__ void begin(const Params& p, int m_row, int nt) {
+    const int v = m_row;
     valid = v < p.V;
     nbase = nt * kBN;
     o = valid ? p.out + static_cast<long long>(v) * p.d : nullptr;
@@ -155,43 +155,26 @@ struct EpiDW {
   __device__ __forceinline__ void end(const Params&) {}
 };
 
-template <bool A_MN, bool B_MN, class Epi>
-static cudaError_t run_gemm(const CUtensorMap& mapA, const CUtensorMap& mapB, const GemmGeom& g,
-                            const typename Epi::Params& p, int grid, const DevCtl& ctl,
-                            cudaStream_t st) {
-  auto kern = k_tc_gemm<A_MN, B_MN, Epi>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       kGemmSmemBytes);
-  if (e != cudaSuccess) return e;
-  const int tiles = g.m_tiles * g.n_tiles;
-  if (tiles == 0) return cudaSuccess;
-  kern<<<grid < tiles ? grid : tiles, kGemmThreads, kGemmSmemBytes, st>>>(mapA, mapB, g, p, ctl);
-  return cudaGetLastError();
-}
-
 cudaError_t launch_bwd_grad(const CUtensorMap& mapA, const CUtensorMap& mapB, int Mc, int V,
                             int d, int tok0, const int* y, const float* lse, const float* coef,
                             const int* rowid, uint16_t* G, long long ldG, int grid,
                             const DevCtl& ctl, cudaStream_t st) {
-  GemmGeom g{(Mc + kBM - 1) / kBM, (V + kBN - 1) / kBN, (d + kBK - 1) / kBK, 0};
   EpiGrad::Params p{y, lse, coef, rowid, G, ldG, Mc, V, tok0};
-  return run_gemm<false, false, EpiGrad>(mapA, mapB, g, p, grid, ctl, st);
+  return launch_gemm<false, false, EpiGrad>(mapA, mapB, Mc, V, d, 0, p, grid, ctl, st);
 }
 
 cudaError_t launch_bwd_dh(const CUtensorMap& mapA, const CUtensorMap& mapB, int Mc, int V, int d,
                           int tok0, const int* dst, float* dH, int grid, const DevCtl& ctl,
                           cudaStream_t st) {
-  GemmGeom g{(Mc + kBM - 1) / kBM, (d + kBN - 1) / kBN, (V + kBK - 1) / kBK, 1};
   EpiRows::Params p{dst, dH, Mc, d, tok0};
-  return run_gemm<false, true, EpiRows>(mapA, mapB, g, p, grid, ctl, st);
+  return launch_gemm<false, true, EpiRows>(mapA, mapB, Mc, d, V, 1, p, grid, ctl, st);
 }
 
 cudaError_t launch_bwd_dw(const CUtensorMap& mapA, const CUtensorMap& mapB, int Mc, int V, int d,
                           float* dW, int accumulate, int grid, const DevCtl& ctl,
                           cudaStream_t st) {
-  GemmGeom g{(V + kBM - 1) / kBM, (d + kBN - 1) / kBN, (Mc + kBK - 1) / kBK, 1};
   EpiDW::Params p{dW, V, d, accumulate};
-  return run_gemm<true, true, EpiDW>(mapA, mapB, g, p, grid, ctl, st);
+  return launch_gemm<true, true, EpiDW>(mapA, mapB, V, d, Mc, 1, p, grid, ctl, st);
 }
 
 }  // namespace dpo

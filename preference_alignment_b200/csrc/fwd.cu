@@ -16,7 +16,7 @@
 #include <cmath>
 
 #include "internal.h"
-#include "tc_gemm.cuh"
+#include "gemm_launch.cuh"
 
 namespace dpo {
 
@@ -90,9 +90,9 @@ struct EpiLSE {
   bool valid;
   float mx, s, zyv;
 
-  __device__ __forceinline__ void begin(const Params& p, int mt, int nt_, int row) {
+  __device__ __forceinline__ void begin(const Params& p, int m_row, int nt_) {
     nt = nt_;
-    tok = mt * kBM + row;
+    tok = m_row;
     valid = tok < p.Nc;
     const int vbase = nt * kBN;
     yl = valid ? __ldg(p.y + tok) - vbase : -1;   // y = -1 (bad target) never matches
@@ -140,50 +140,71 @@ cudaError_t launch_fwd_lse(const CUtensorMap& mapA, const CUtensorMap& mapB, int
                            int d, const int* y, float2* part, int ldp, float* zy, int grid,
                            const DevCtl& ctl, cudaStream_t st) {
   if (Nc == 0) return cudaSuccess;
-  GemmGeom g;
-  g.m_tiles = (Nc + kBM - 1) / kBM;
-  g.n_tiles = (V + kBN - 1) / kBN;
-  g.k_blocks = (d + kBK - 1) / kBK;
-  g.order = 0;
   EpiLSE::Params p{y, part, zy, Nc, V, ldp};
-  auto kern = k_tc_gemm<false, false, EpiLSE>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       kGemmSmemBytes);
-  if (e != cudaSuccess) return e;
-  const int tiles = g.m_tiles * g.n_tiles;
-  kern<<<grid < tiles ? grid : tiles, kGemmThreads, kGemmSmemBytes, st>>>(mapA, mapB, g, p, ctl);
-  return cudaGetLastError();
+  // order 0: all token tiles of one vocab tile run together, so each W tile is
+  // read from HBM once and served to the other CTAs from L2
+  return launch_gemm<false, false, EpiLSE>(mapA, mapB, Nc, V, d, 0, p, grid, ctl, st);
 }
 
 // ------------------------------------------------------------------ combine
-// lse_i = M + log(sum_s s_s * exp(m_s - M)), accumulated over vocab tiles in
-// increasing order (deterministic), then lp_i = z_y - lse_i.
+// lse_i = M + log(sum_s s_s * exp(m_s - M)) over the vocab-tile partials of
+// position i, then lp_i = z_y - lse_i. A block covers 32 positions; its 8 warps
+// take the partials s = g, g + 8, ... (warp g), reading 32 consecutive positions
+// per partial (coalesced), and the 8 running (max, sum) pairs are merged in warp
+// order. The assignment and the merge order are fixed, so the result is
+// bit-identical from run to run.
+__device__ __forceinline__ void lse_merge(float& M, float& S, float m, float s) {
+  if (m == -INFINITY) return;
+  if (m > M) {
+    S = S * expf(M - m) + s;
+    M = m;
+  } else {
+    S += s * expf(m - M);
+  }
+}
+
 __global__ void __launch_bounds__(256) k_combine(const float2* __restrict__ part, int ldp, int S,
                                                  const float* __restrict__ zy,
                                                  const int* __restrict__ y, int Nc,
                                                  float* __restrict__ lp,
                                                  float* __restrict__ lse_out) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= Nc) return;
+  __shared__ float sm[8][32], ss[8][32];
+  const int g = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int i = blockIdx.x * 32 + lane;
   float M = -INFINITY, sum = 0.f;
-  for (int s = 0; s < S; ++s) {
-    const float2 q = __ldg(part + static_cast<long long>(s) * ldp + i);
-    if (q.x > M) {
-      sum = sum * expf(M - q.x) + q.y;
-      M = q.x;
-    } else {
-      sum += q.y * expf(q.x - M);
+  if (i < Nc) {
+    int s = g;
+    for (; s + 24 < S; s += 32) {          // four independent loads in flight
+      const float2 q0 = __ldg(part + static_cast<long long>(s) * ldp + i);
+      const float2 q1 = __ldg(part + static_cast<long long>(s + 8) * ldp + i);
+      const float2 q2 = __ldg(part + static_cast<long long>(s + 16) * ldp + i);
+      const float2 q3 = __ldg(part + static_cast<long long>(s + 24) * ldp + i);
+      lse_merge(M, sum, q0.x, q0.y);
+      lse_merge(M, sum, q1.x, q1.y);
+      lse_merge(M, sum, q2.x, q2.y);
+      lse_merge(M, sum, q3.x, q3.y);
+    }
+    for (; s < S; s += 8) {
+      const float2 q = __ldg(part + static_cast<long long>(s) * ldp + i);
+      lse_merge(M, sum, q.x, q.y);
     }
   }
-  const float lse = M + logf(sum);
-  lp[i] = (__ldg(y + i) >= 0) ? __ldg(zy + i) - lse : 0.f;
-  if (lse_out != nullptr) lse_out[i] = lse;
+  sm[g][lane] = M;
+  ss[g][lane] = sum;
+  __syncthreads();
+  if (g == 0 && i < Nc) {
+    float Mt = sm[0][lane], St = ss[0][lane];
+    for (int h = 1; h < 8; ++h) lse_merge(Mt, St, sm[h][lane], ss[h][lane]);
+    const float lse = Mt + logf(St);
+    lp[i] = (__ldg(y + i) >= 0) ? __ldg(zy + i) - lse : 0.f;
+    if (lse_out != nullptr) lse_out[i] = lse;
+  }
 }
 
 cudaError_t launch_combine(const float2* part, int ldp, int S, const float* zy, const int* y,
                            int Nc, float* lp, float* lse_out, cudaStream_t st) {
   if (Nc == 0) return cudaSuccess;
-  k_combine<<<(Nc + 255) / 256, 256, 0, st>>>(part, ldp, S, zy, y, Nc, lp, lse_out);
+  k_combine<<<(Nc + 31) / 32, 256, 0, st>>>(part, ldp, S, zy, y, Nc, lp, lse_out);
   return cudaGetLastError();
 }
 

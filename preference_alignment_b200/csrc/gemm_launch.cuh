@@ -1,0 +1,65 @@
+// Host-side launch of the tcgen05 GEMM kernels (included by the .cu files that
+// instantiate them). The CTA-pair kernel is the default; the single-CTA kernel
+// is used when the device cannot co-schedule CTA pairs.
+#pragma once
+
+#include "tc_gemm.cuh"
+
+namespace dpo {
+
+// Clusters of two that can be resident at once for a pair-kernel instantiation
+// on the current device (cached per device).
+template <class Kern>
+int max_pair_clusters(Kern kern, int smem_bytes) {
+  static int cache[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  if (cache[dev] != 0) return cache[dev] > 0 ? cache[dev] : 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2, 1, 1);
+  cfg.blockDim = dim3(kGemmThreads, 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem_bytes);
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+    (void)cudaGetLastError();
+    n = 0;
+  }
+  cache[dev] = n > 0 ? n : -1;
+  return n;
+}
+
+// D[M x N] = A[M x K] . B[N x K]^T with the epilogue Epi; `order` picks the tile
+// raster (0: M fastest, 1: N fastest); `sms` is the device's SM count.
+template <bool A_MN, bool B_MN, class Epi>
+cudaError_t launch_gemm(const CUtensorMap& mapA, const CUtensorMap& mapB, int M, int N, int K,
+                        int order, const typename Epi::Params& p, int sms, const DevCtl& ctl,
+                        cudaStream_t st) {
+  const int n_tiles = (N + kBN - 1) / kBN;
+  const int k_blocks = (K + kBK - 1) / kBK;
+  {
+    auto kern = k_tc_gemm_pair<A_MN, B_MN, Epi>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kPairSmemBytes);
+    if (e != cudaSuccess) return e;
+    const int clusters = max_pair_clusters(kern, kPairSmemBytes);
+    if (clusters > 0) {
+      GemmGeom g{(M + kPairM - 1) / kPairM, n_tiles, k_blocks, order};
+      const int tiles = g.m_tiles * g.n_tiles;
+      int pairs = clusters < sms / 2 ? clusters : sms / 2;
+      if (pairs > tiles) pairs = tiles;
+      if (pairs < 1) pairs = 1;
+      kern<<<2 * pairs, kGemmThreads, kPairSmemBytes, st>>>(mapA, mapB, g, p, ctl);
+      return cudaGetLastError();
+    }
+  }
+  auto kern = k_tc_gemm<A_MN, B_MN, Epi>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       kGemmSmemBytes);
+  if (e != cudaSuccess) return e;
+  GemmGeom g{(M + kBM - 1) / kBM, n_tiles, k_blocks, order};
+  const int tiles = g.m_tiles * g.n_tiles;
+  kern<<<sms < tiles ? sms : tiles, kGemmThreads, kGemmSmemBytes, st>>>(mapA, mapB, g, p, ctl);
+  return cudaGetLastError();
+}
+
+}  // namespace dpo

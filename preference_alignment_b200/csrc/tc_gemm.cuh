@@ -49,7 +49,7 @@ __device__ __forceinline__ void tile_coords(const GemmGeom& g, int tile, int& mt
 }
 
 // Epilogue interface (one object per epilogue thread, per tile):
-//   __device__ void begin(const Params&, int mt, int nt, int row);
+//   __device__ void begin(const Params&, int m_row, int nt);   // m_row: absolute row of D
 //   __device__ void chunk(const Params&, int c, const uint32_t (&v)[32]);   // columns c*32..+31
 //   __device__ void end(const Params&);
 template <bool A_MN, bool B_MN, class Epi>
@@ -132,7 +132,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             tma_load_2d(a_dst + j * 8192, &tmA, fb, mt * kBM + j * 64, kb * kBK);
         }
         if (!B_MN) {
+          // two 128-row boxes: the same tensor map serves the CTA-pair kernel
           tma_load_2d(b_dst, &tmB, fb, kb * kBK, nt * kBN);
+          tma_load_2d(b_dst + 128 * 128, &tmB, fb, kb * kBK, nt * kBN + 128);
         } else {
 #pragma unroll
           for (int j = 0; j < kBN / 64; ++j)
@@ -221,7 +223,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int mt, nt;
       tile_coords(g, tile, mt, nt);
       Epi epi;
-      epi.begin(ep, mt, nt, row);
+      epi.begin(ep, mt * kBM + row, nt);
 #pragma unroll 1
       for (int c = 0; c < kBN / 32; ++c) {
         uint32_t v[32];
@@ -253,6 +255,219 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+
+// =====================================================================================
+// Pair variant: two CTAs of a cluster compute a 256 x 256 tile with
+// tcgen05.mma.cta_group::2 (M = 256 across the pair). Each CTA loads its own 128
+// rows of A and its own 128 rows (N half) of B, so a CTA moves 32 KiB per K step
+// instead of 48 KiB; the freed shared memory buys a 6-deep pipeline.
+//   leader (cluster rank 0): owns the `full` and `acc_empty` barriers and issues
+//     the MMAs; its commits are multicast to both CTAs' `empty` / `acc_full`.
+//   both CTAs: TMA producer, epilogue over their own 128 TMEM lanes (rows
+//     rank * 128 ... + 127 of the 256-row tile), arriving on the leader's
+//     `acc_empty` through its shared::cluster address.
+// No TMA load uses cluster multicast: each CTA reads only its own operand rows.
+// =====================================================================================
+constexpr int kPairM = 256;                        // rows of D per CTA pair
+constexpr int kPStages = 6;
+constexpr int kPABytes = 128 * kBK * 2;            // 16 KiB: this CTA's 128 rows of A
+constexpr int kPBBytes = (kBN / 2) * kBK * 2;      // 16 KiB: this CTA's half of B
+constexpr int kPStageBytes = kPABytes + kPBBytes;
+constexpr int kPairSmemBytes = kPStages * kPStageBytes + 1024 + 256;
+
+template <bool A_MN, bool B_MN, class Epi>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
+    k_tc_gemm_pair(const __grid_constant__ CUtensorMap tmA,
+                   const __grid_constant__ CUtensorMap tmB, GemmGeom g,
+                   typename Epi::Params ep, DevCtl ctl) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + kPStages * kPABytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kPStages * kPStageBytes);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kPStages + 5);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const uint32_t full0 = smem_u32(bars);
+  const uint32_t empty0 = smem_u32(bars + kPStages);
+  const uint32_t accf0 = smem_u32(bars + 2 * kPStages);
+  const uint32_t acce0 = smem_u32(bars + 2 * kPStages + 2);
+  const uint32_t drain = smem_u32(bars + 2 * kPStages + 4);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kPStages; ++s) {
+      mbar_init(full0 + 8 * s, 1);          // leader: its arrive.expect_tx (both CTAs' bytes)
+      mbar_init(empty0 + 8 * s, 1);         // one multicast commit per phase
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(accf0 + 8 * a, 1);
+      mbar_init(acce0 + 8 * a, 2 * 128);    // leader: every epilogue thread of both CTAs
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync_all();                       // barriers initialised in both CTAs
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int pair = blockIdx.x >> 1;
+  const int n_pairs = gridDim.x >> 1;
+  const int n_tiles_total = g.m_tiles * g.n_tiles;   // m_tiles counts 256-row tiles
+
+  if (warp == 0 && lane == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    const uint32_t full_leader = mapa_shared(full0, 0);
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int tile = pair; tile < n_tiles_total && ok; tile += n_pairs) {
+      int mt, nt;
+      tile_coords(g, tile, mt, nt);
+      const int arow = mt * kPairM + static_cast<int>(rank) * 128;
+      const int brow = nt * kBN + static_cast<int>(rank) * (kBN / 2);
+      for (int kb = 0; kb < g.k_blocks; ++kb) {
+        if (!mbar_wait(empty0 + 8 * stage, phase ^ 1, ctl, abort_flag)) {
+          ok = false;
+          break;
+        }
+        if (leader) mbar_arrive_expect_tx(full0 + 8 * stage, 2 * kPStageBytes);
+        const uint32_t fb = full_leader + 8 * stage;
+        const uint32_t a_dst = smem_u32(sA + stage * kPABytes);
+        const uint32_t b_dst = smem_u32(sB + stage * kPBBytes);
+        if (!A_MN) {
+          tma_load_2d_pair(a_dst, &tmA, fb, kb * kBK, arow);
+        } else {
+          tma_load_2d_pair(a_dst, &tmA, fb, arow, kb * kBK);
+          tma_load_2d_pair(a_dst + 8192, &tmA, fb, arow + 64, kb * kBK);
+        }
+        if (!B_MN) {
+          tma_load_2d_pair(b_dst, &tmB, fb, kb * kBK, brow);
+        } else {
+          tma_load_2d_pair(b_dst, &tmB, fb, brow, kb * kBK);
+          tma_load_2d_pair(b_dst + 8192, &tmB, fb, brow + 64, kb * kBK);
+        }
+        if (++stage == kPStages) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+    }
+    if (!ok) {
+      record_status(ctl, kStatusTimeout);
+      *abort_flag = 1;
+    }
+  } else if (warp == 1 && lane == 0 && leader) {
+    // ---------------------------------------------------------------- MMA issuer (leader)
+    constexpr uint32_t idesc = idesc_bf16_f32(kPairM, kBN, A_MN, B_MN);
+    int stage = 0;
+    uint32_t phase = 0;
+    int local = 0;
+    bool ok = true;
+    for (int tile = pair; tile < n_tiles_total && ok; tile += n_pairs, ++local) {
+      const int acc = local & 1;
+      const uint32_t acc_phase = (local >> 1) & 1;
+      if (!mbar_wait(acce0 + 8 * acc, acc_phase ^ 1, ctl, abort_flag)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + acc * kBN;
+      for (int kb = 0; kb < g.k_blocks; ++kb) {
+        if (!mbar_wait(full0 + 8 * stage, phase, ctl, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a0 = smem_u32(sA + stage * kPABytes);
+        const uint32_t b0 = smem_u32(sB + stage * kPBBytes);
+#pragma unroll
+        for (int k = 0; k < kBK / 16; ++k) {
+          const uint64_t ad = A_MN ? sw128_desc(a0 + k * 2048, 8192, 1024)
+                                   : sw128_desc(a0 + k * 32, 16, 1024);
+          const uint64_t bd = B_MN ? sw128_desc(b0 + k * 2048, 8192, 1024)
+                                   : sw128_desc(b0 + k * 32, 16, 1024);
+          tc_mma_f16_pair(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
+        }
+        tc_commit_pair_mc(empty0 + 8 * stage, 0x3);
+        if (++stage == kPStages) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+      if (!ok) break;
+      tc_commit_pair_mc(accf0 + 8 * acc, 0x3);
+    }
+    if (!ok) {
+      record_status(ctl, kStatusTimeout);
+      *abort_flag = 1;
+    }
+    tc_commit_pair(drain);
+    volatile int never = 0;
+    if (!mbar_wait(drain, 0, ctl, &never)) record_status(ctl, kStatusTimeout);
+  } else if (warp >= 2) {
+    // ---------------------------------------------------------------- epilogue (both CTAs)
+    const int lg = warp & 3;
+    const int row = static_cast<int>(rank) * 128 + lg * 32 + lane;
+    const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(lg * 32) << 16);
+    const uint32_t acce_leader = mapa_shared(acce0, 0);
+    int local = 0;
+    for (int tile = pair; tile < n_tiles_total; tile += n_pairs, ++local) {
+      const int acc = local & 1;
+      const uint32_t acc_phase = (local >> 1) & 1;
+      if (!mbar_wait(accf0 + 8 * acc, acc_phase, ctl, abort_flag)) {
+        record_status(ctl, kStatusTimeout);
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      int mt, nt;
+      tile_coords(g, tile, mt, nt);
+      Epi epi;
+      epi.begin(ep, mt * kPairM + row, nt);
+#pragma unroll 1
+      for (int c = 0; c < kBN / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(lane_addr + acc * kBN + c * 32, v);
+        tmem_wait_ld();
+        epi.chunk(ep, c, v);
+      }
+      tc_fence_before();
+      mbar_arrive_cluster(acce_leader + 8 * acc);
+      epi.end(ep);
+    }
+  }
+
+  // ---------------------------------------------------------------- teardown
+  __syncthreads();
+  if (threadIdx.x == 0 && *abort_flag) {
+    // After an abort a load issued just before may still be landing in this CTA's
+    // shared memory: give it a bounded 2 ms before the pair leaves.
+    const unsigned long long t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < 2000000ull) {
+    }
+  }
+  tc_fence_before();
+  cluster_sync_all();                       // neither CTA leaves while the pair is in use
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc_pair(tmem_base, kTmemCols);
   }
 }
 
