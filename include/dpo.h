@@ -144,6 +144,30 @@ dpo_status dpo_backward(const dpo_batch* batch, const float* lse_state, const fl
                         float* dH, float* dW, int accumulate_dW, void* ws, size_t ws_bytes,
                         void* stream);
 
+/* Size of the scratch array built into the library for dpo_seq_logprobs_noalloc. */
+#define DPO_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+/* dpo_seq_logprobs without a workspace argument, for callers that may not
+ * allocate device memory (for example code running inside a framework that owns
+ * the device-memory budget and forbids allocation from its plugins, or code that
+ * cannot accept the device-wide synchronisation cudaMalloc/cudaFree may cause).
+ * The pages have no counterpart: this is a deployment convenience of the library.
+ *   Arguments, outputs and errors are those of dpo_seq_logprobs.
+ *   Scratch: a DPO_NOALLOC_SCRATCH_BYTES (32 MiB) array compiled into the
+ *   library, held by every device that loads it until the process exits. A batch
+ *   whose forward workspace (dpo_workspace_size's fwd_bytes) exceeds that size is
+ *   refused with DPO_ERR_WORKSPACE before any device work.
+ *   Set-up: the first call on a device, made with that device current, looks the
+ *   array's address up (cudaGetSymbolAddress); make that first call before any
+ *   stream capture.
+ *   Sharing: all calls on a device use the same array and it keeps the last
+ *   call's contents (every byte a call reads is written by that call first).
+ *   Calls whose work overlaps on the GPU (different streams, or different host
+ *   threads without ordering) race on the array: serialise them.
+ *   The call allocates no device memory. */
+dpo_status dpo_seq_logprobs_noalloc(const dpo_batch* batch, int want_grad, float* seq_logp,
+                                    float* tok_logp, float* lse_state, void* stream);
+
 /* Synchronise `stream`, then return and clear the current device's status word
  * (DPO_OK, DPO_ERR_TIMEOUT or DPO_ERR_BAD_TARGET), or DPO_ERR_CUDA if the
  * synchronisation itself failed. */

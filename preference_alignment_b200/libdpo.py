@@ -186,3 +186,23 @@ def backward(batch: BatchArgs, lse_state, row_coef, dH, dW, accumulate_dW: bool,
 def check(stream=None) -> int:
     """Synchronise the stream and return (and clear) the device status word."""
     return load().dpo_check(_stream(stream))
+
+
+def seq_logprobs_noalloc(batch: BatchArgs, want_grad: bool, seq_logp, tok_logp, lse_state,
+                         stream=None):
+    """dpo_seq_logprobs_noalloc: the forward with the library's built-in scratch.
+
+    For callers that may not allocate device memory (no workspace argument). The
+    batch's forward workspace must fit NOALLOC_SCRATCH_BYTES; calls that overlap on
+    the GPU share the scratch and must be serialised.
+    """
+    lib = load()
+    fn = lib.dpo_seq_logprobs_noalloc
+    fn.argtypes = [ctypes.POINTER(Batch), ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
+                   ctypes.c_void_p, ctypes.c_void_p]
+    fn.restype = ctypes.c_int
+    _check(fn(ctypes.byref(batch.c), 1 if want_grad else 0, _ptr(seq_logp), _ptr(tok_logp),
+              _ptr(lse_state), _stream(stream)), "dpo_seq_logprobs_noalloc")
+
+
+NOALLOC_SCRATCH_BYTES = 32 << 20
