@@ -66,7 +66,7 @@ def rank_workload(name, rank):
     w.prompt_len = P.astype(np.int32)
     w.completion_len = C.astype(np.int32)
     w.tokens = rng.integers(0, V, size=(R, L), dtype=np.int64).astype(np.int32)
-    w.H = WL.bf16_bits_from_f32(rng.standard_normal(size=(R, L, d), dtype=np.float32))
+    w.H = WL.encode(rng.standard_normal(size=(R, L, d), dtype=np.float32), w.dtype)
     return w
 
 
@@ -215,6 +215,7 @@ def run_ours(args):
     import torch
     import torch.distributed as dist
 
+    from preference_alignment_b200 import dp as DP
     from preference_alignment_b200 import libdpo
 
     ws_n, rank, local = dist_env()
@@ -252,7 +253,7 @@ def run_ours(args):
              ("coef", 2 * B)]}
     stream = torch.cuda.current_stream(dev)
     sp = stream.cuda_stream
-    grad_scale = 1.0 / ws_n                  # loss is the mean over the global batch
+    grad_scale = DP.grad_scale(ws_n)         # loss is the mean over the global batch
 
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
 
@@ -283,10 +284,8 @@ def run_ours(args):
             ev[4].record(stream)
             torch.cuda.synchronize(dev)
             timed.append([ev[i].elapsed_time(ev[i + 1]) for i in range(4)])
-        if ws_n > 1:
-            dist.all_reduce(dW)
-            dist.all_reduce(outs["loss"])
-            outs["loss"].mul_(1.0 / ws_n)
+        if ws_n > 1 and not fwd_only:
+            DP.allreduce_step(dW, outs["loss"])
 
     # launches of our kernels per step: upload + prep + GEMM + combine + rowsum per forward,
     # one loss kernel, upload + prep + 3 GEMMs for the backward (one token chunk: the

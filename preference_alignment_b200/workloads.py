@@ -87,8 +87,12 @@ def _normal(rng, shape, std, dtype):
     return x
 
 
-def _encode(x: np.ndarray, dtype: str) -> np.ndarray:
+def encode(x: np.ndarray, dtype: str) -> np.ndarray:
+    """Stored form of float32 draws: bf16 bit patterns (rounded) or float32 values."""
     return bf16_bits_from_f32(x) if dtype == "bf16" else np.ascontiguousarray(x, np.float32)
+
+
+_encode = encode
 
 
 def _draw_common(rng, R, L, d, V, dtype, ref_std, P, C, with_ref=True):

@@ -1,0 +1,144 @@
+"""The C ABI on a machine without a GPU: the library loads, exports every entry
+point include/dpo.h declares, and rejects bad arguments on the host before any
+CUDA call (errors leave outputs untouched and need no device)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from preference_alignment_b200 import build as B
+from preference_alignment_b200 import libdpo
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dpo.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return libdpo.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(dpo_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for n in ("dpo_workspace_size", "dpo_seq_logprobs", "dpo_loss", "dpo_backward", "dpo_check",
+              "dpo_status_string", "dpo_version", "dpo_set_wait_budget_ms"):
+        assert n in names
+    text = open(HEADER).read()
+    assert "torch" not in re.sub(r"/\*.*?\*/", "", text, flags=re.S).lower()
+    assert 'extern "C"' in text
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for n in declared_functions():
+        assert hasattr(lib, n), f"{n} is declared in dpo.h but not exported"
+
+
+def test_status_strings_and_version(lib):
+    for code in range(7):
+        assert libdpo.status_string(code)
+    assert libdpo.status_string(99) == "unknown status"
+    assert libdpo.version() == 100
+
+
+FAKE = 0x10000  # never dereferenced: every call below fails its host checks first
+
+
+def _batch(R=4, L=32, d=64, V=100, dtype="bf16", P=None, C=None, H=FAKE, W=FAKE, tokens=FAKE):
+    P = np.full(R, 4, np.int32) if P is None else np.asarray(P, np.int32)
+    C = np.full(R, 10, np.int32) if C is None else np.asarray(C, np.int32)
+    return libdpo.BatchArgs(H, W, tokens, P, C, R=R, L=L, d=d, V=V, dtype=dtype)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(dtype="f16"), libdpo.ERR_UNSUPPORTED),          # fp16 refused
+    (dict(dtype=7), libdpo.ERR_INVALID_ARG),
+    (dict(d=60), libdpo.ERR_UNSUPPORTED),                  # d must be a multiple of 8
+    (dict(R=0), libdpo.ERR_INVALID_ARG),
+    (dict(L=1), libdpo.ERR_INVALID_ARG),
+    (dict(V=0), libdpo.ERR_INVALID_ARG),
+    (dict(V=(1 << 24) + 1), libdpo.ERR_INVALID_ARG),
+    (dict(P=[0, 4, 4, 4]), libdpo.ERR_INVALID_ARG),        # no predictor for the first token
+    (dict(C=[-1, 10, 10, 10]), libdpo.ERR_INVALID_ARG),
+    (dict(P=[20, 4, 4, 4], C=[13, 10, 10, 10]), libdpo.ERR_INVALID_ARG),  # P + C > L
+    (dict(H=FAKE + 8), libdpo.ERR_INVALID_ARG),            # H not 16-byte aligned
+    (dict(W=0), libdpo.ERR_INVALID_ARG),                   # null W
+])
+def test_workspace_size_rejects(lib, kw, code):
+    with pytest.raises(libdpo.DpoError) as e:
+        libdpo.workspace_size(_batch(**kw))
+    assert e.value.status == code
+
+
+def test_workspace_sizes_are_consistent(lib):
+    f1, b1, m1 = libdpo.workspace_size(_batch())
+    assert f1 % 256 == 0 and b1 % 256 == 0 and m1 % 256 == 0
+    assert m1 <= b1
+    # more scored positions never need less
+    f2, b2, m2 = libdpo.workspace_size(_batch(C=[20, 20, 20, 20]))
+    assert f2 >= f1 and b2 >= b1
+    # the backward workspace grows with Nc * V (the bf16 dz chunk), the forward with Nc * d
+    f3, b3, _ = libdpo.workspace_size(_batch(V=10000))
+    assert b3 - b1 >= 40 * (10000 - 100) * 2 * 0.99
+    # an empty batch still gets a valid, small workspace
+    f0, b0, m0 = libdpo.workspace_size(_batch(C=[0, 0, 0, 0]))
+    assert 0 < f0 <= f1 and 0 < m0 <= b0
+
+
+def test_calls_fail_on_the_host_and_leave_outputs_alone(lib):
+    out = np.full(4, 7.0, np.float32)      # host array: must never be written
+    b = _batch(P=[0, 4, 4, 4])
+    with pytest.raises(libdpo.DpoError) as e:
+        libdpo.seq_logprobs(b, False, out, None, None, FAKE, ws_bytes=1 << 30)
+    assert e.value.status == libdpo.ERR_INVALID_ARG
+    b = _batch()
+    with pytest.raises(libdpo.DpoError) as e:   # no workspace
+        libdpo.seq_logprobs(b, False, out, None, None, 0, ws_bytes=0)
+    assert e.value.status == libdpo.ERR_WORKSPACE
+    with pytest.raises(libdpo.DpoError) as e:   # misaligned workspace
+        libdpo.seq_logprobs(b, False, out, None, None, FAKE + 16, ws_bytes=1 << 30)
+    assert e.value.status == libdpo.ERR_WORKSPACE
+    with pytest.raises(libdpo.DpoError) as e:   # want_grad without lse_state
+        libdpo.seq_logprobs(b, True, out, None, None, FAKE, ws_bytes=1 << 30)
+    assert e.value.status == libdpo.ERR_INVALID_ARG
+    with pytest.raises(libdpo.DpoError) as e:   # backward without dW
+        libdpo.backward(b, FAKE, FAKE, None, None, False, FAKE, ws_bytes=1 << 30)
+    assert e.value.status == libdpo.ERR_INVALID_ARG
+    f, bw, mn = libdpo.workspace_size(b)
+    with pytest.raises(libdpo.DpoError) as e:   # backward workspace below the minimum
+        libdpo.backward(b, FAKE, FAKE, None, FAKE, False, FAKE, ws_bytes=mn - 256)
+    assert e.value.status == libdpo.ERR_WORKSPACE
+    assert np.all(out == 7.0)
+
+
+@pytest.mark.parametrize("args", [
+    dict(B=0), dict(layout=2), dict(beta=0.0), dict(beta=-1.0), dict(beta=float("nan")),
+    dict(grad_scale=float("inf")), dict(pol=None), dict(loss_out=None),
+])
+def test_loss_rejects(lib, args):
+    a = dict(B=2, layout="halves", pol=FAKE, ref=FAKE, beta=0.1, grad_scale=1.0, loss_out=FAKE)
+    a.update(args)
+    with pytest.raises(libdpo.DpoError) as e:
+        libdpo.loss(a["B"], a["layout"], a["pol"], a["ref"], a["beta"], a["grad_scale"],
+                    a["loss_out"])
+    assert e.value.status == libdpo.ERR_INVALID_ARG
+
+
+def test_noalloc_refuses_oversized_batches_on_the_host(lib):
+    b = _batch(R=2, L=4096, d=4096, V=1000, P=[1, 1], C=[4095, 4095])
+    with pytest.raises(libdpo.DpoError) as e:
+        libdpo.seq_logprobs_noalloc(b, False, FAKE, None, None)
+    assert e.value.status == libdpo.ERR_WORKSPACE
+
+
+def test_wait_budget_roundtrip(lib):
+    old = libdpo.set_wait_budget_ms(1234)
+    assert libdpo.set_wait_budget_ms(old) == 1234
