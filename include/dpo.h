@@ -14,9 +14,10 @@
  *  dpo_step in "A training configuration that fits".)
  *
  * Conventions shared by every call
- *   - Every buffer is owned by the caller. The library allocates no device
- *     memory; each call that needs scratch takes a caller-provided workspace
- *     whose size dpo_workspace_size() returns.
+ *   - Every buffer is owned by the caller. The library makes no device-memory
+ *     allocation calls; each call that needs scratch takes a caller-provided
+ *     workspace whose size dpo_workspace_size() returns (the one exception,
+ *     dpo_seq_logprobs_noalloc, uses a scratch array compiled into the library).
  *   - Device pointers must point to device memory of the current CUDA device.
  *     "host" marks the few arguments read from host memory during the call.
  *   - `stream` is a cudaStream_t (NULL = the legacy default stream). All device
@@ -173,11 +174,19 @@ dpo_status dpo_seq_logprobs_noalloc(const dpo_batch* batch, int want_grad, float
  * synchronisation itself failed. */
 dpo_status dpo_check(void* stream);
 
-/* Time budget, in milliseconds, of every bounded wait inside the kernels of the
- * calling host thread's current device (default 4000). A wait that exceeds it
+/* Time budget, in milliseconds, of every bounded wait inside the kernels
+ * launched afterwards by this process (default 4000). A wait that exceeds it
  * makes the kernel record DPO_ERR_TIMEOUT, drain its in-flight copies and MMAs
  * (again bounded) and exit. Returns the previous value. */
 uint32_t dpo_set_wait_budget_ms(uint32_t ms);
+
+/* Self-test of the kernels' bounded waits: launches one CTA that waits, with the
+ * same bounded wait the GEMM pipelines use, on a barrier nothing ever arrives on.
+ * After budget_ms the wait gives up and records DPO_ERR_TIMEOUT in the status
+ * word, which the next dpo_check(stream) returns; the kernel exits normally and
+ * the context stays usable. No counterpart on the pages: a diagnostic of this
+ * library's failure handling. */
+dpo_status dpo_selftest_wait_timeout(uint32_t budget_ms, void* stream);
 
 /* Static description of a status code. */
 const char* dpo_status_string(dpo_status s);

@@ -369,6 +369,15 @@ dpo_status dpo_check(void* stream) {
   return static_cast<dpo_status>(v);
 }
 
+dpo_status dpo_selftest_wait_timeout(uint32_t budget_ms, void* stream) {
+  DevInfo di;
+  dpo_status s = device_info(&di);
+  if (s != DPO_OK) return s;
+  DevCtl ctl = make_ctl(di);
+  ctl.budget_ns = static_cast<unsigned long long>(budget_ms < 1 ? 1 : budget_ms) * 1000000ull;
+  return cuda_status(launch_wait_selftest(ctl, static_cast<cudaStream_t>(stream)));
+}
+
 uint32_t dpo_set_wait_budget_ms(uint32_t ms) { return g_budget_ms.exchange(ms < 1 ? 1 : ms); }
 
 const char* dpo_status_string(dpo_status s) {

@@ -183,6 +183,15 @@ def backward(batch: BatchArgs, lse_state, row_coef, dH, dW, accumulate_dW: bool,
                                _nbytes(ws, ws_bytes), _stream(stream)), "dpo_backward")
 
 
+def selftest_wait_timeout(budget_ms: int, stream=None):
+    """Launch the bounded-wait self-test (records DPO_ERR_TIMEOUT after budget_ms)."""
+    lib = load()
+    fn = lib.dpo_selftest_wait_timeout
+    fn.argtypes = [ctypes.c_uint32, ctypes.c_void_p]
+    fn.restype = ctypes.c_int
+    _check(fn(int(budget_ms), _stream(stream)), "dpo_selftest_wait_timeout")
+
+
 def check(stream=None) -> int:
     """Synchronise the stream and return (and clear) the device status word."""
     return load().dpo_check(_stream(stream))
