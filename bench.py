@@ -55,9 +55,17 @@ def dist_env():
     return ws, rank, local
 
 
-def rank_workload(name, rank):
-    """The named workload with this rank's own batch (same weights on every rank)."""
-    w = WL.make_config(name)
+def rank_workload(name, rank, weights=True):
+    """The named workload with this rank's own batch (same weights on every rank).
+
+    With weights=False a rank > 0 draws only its batch (W and W_ref are None) and
+    receives the weights from rank 0."""
+    if rank > 0 and not weights:
+        idx, R, L, d, V, dtype, layout, ref_std, rule, has_ref = WL.CONFIGS[name]
+        w = WL.Workload(name, R, L, d, V, dtype, layout, 0.1, None, None, None, None, None, None,
+                        WL.SEED_BASE + idx)
+    else:
+        w = WL.make_config(name)
     if rank == 0:
         return w
     idx, R, L, d, V, dtype, layout, ref_std, rule, _ = WL.CONFIGS[name]
@@ -118,6 +126,68 @@ class ClockSampler:
         sm = [r[0] for r in rows]
         return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": max(r[1] for r in rows),
                 "samples": len(rows), "reasons": reasons}
+
+
+def cublas_sustained(torch, dev, stream, seconds=1.5, n=8192):
+    """bf16 torch.matmul (cuBLAS) back to back for `seconds`: TFLOP/s and the SM clock seen.
+
+    Context only (same GPU, same moment); the roofline uses MEASURED_PEAKS.json."""
+    a = torch.randn(n, n, device=dev, dtype=torch.bfloat16)
+    b = torch.randn(n, n, device=dev, dtype=torch.bfloat16)
+    c = torch.empty(n, n, device=dev, dtype=torch.bfloat16)
+    for _ in range(3):
+        torch.matmul(a, b, out=c)
+    torch.cuda.synchronize(dev)
+    sampler = ClockSampler(dev.index)
+    sampler.start()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    iters, t0 = 0, time.perf_counter()
+    e0.record(stream)
+    while time.perf_counter() - t0 < seconds:
+        for _ in range(10):
+            torch.matmul(a, b, out=c)
+        iters += 10
+        torch.cuda.synchronize(dev)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    clk = sampler.stop()
+    ms = e0.elapsed_time(e1)
+    del a, b, c
+    return {"tflops": 2.0 * n ** 3 * iters / (ms / 1e3) / 1e12, "n": n, "seconds": ms / 1e3,
+            "sm_mhz": clk["sm_mhz"] if clk else None,
+            "note": "torch.matmul bf16, same GPU, after the timed regions; context only"}
+
+
+PROFILED_SOURCES = ["preference_alignment_b200/csrc/" + f for f in
+                    ("tc_gemm.cuh", "gemm_launch.cuh", "ptx_sm100.cuh", "tile_config.h", "fwd.cu")]
+
+
+def kernel_source_hash():
+    import hashlib
+    h = hashlib.sha256()
+    for f in PROFILED_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload):
+    """DRAM bytes per launch of the forward GEMM from the committed ncu summary, if the
+    kernel sources are unchanged since the counters were taken (else None)."""
+    path = os.path.join(ROOT, "profiles", f"fwd_lse_gemm_{workload}_dram.md")
+    try:
+        vals = {}
+        with open(path) as f:
+            for line in f:
+                if ":" in line and line.startswith("- "):
+                    k, v = line[2:].split(":", 1)
+                    vals[k.strip()] = v.strip().strip("`")
+        if vals.get("source-hash") != kernel_source_hash():
+            return None
+        return float(vals["dram-bytes-per-launch"])
+    except Exception:
+        return None
 
 
 # ------------------------------------------------------------------ oracle sample (host cores)
@@ -227,16 +297,25 @@ def run_ours(args):
                                 device_id=dev)
     libdpo.load()
 
-    w = rank_workload(args.workload, rank)
+    w = rank_workload(args.workload, rank, weights=(ws_n == 1 or rank == 0))
     B = w.R // 2
 
     def dev_bf16(a):
         return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
 
+    fwd_only = not WL.CONFIGS[args.workload][9]   # offline reference scoring: forward only
     H = dev_bf16(w.H)
-    W = dev_bf16(w.W)
-    fwd_only = w.W_ref is None               # offline reference scoring: forward only
-    Wr = dev_bf16(w.W_ref) if not fwd_only else None
+    if ws_n > 1:
+        # rank 0 drew the weights; the other ranks receive them (same model on every rank)
+        W = dev_bf16(w.W) if rank == 0 else torch.empty(w.V, w.d, dtype=torch.bfloat16, device=dev)
+        dist.broadcast(W, 0)
+        Wr = None
+        if not fwd_only:
+            Wr = dev_bf16(w.W_ref) if rank == 0 else torch.empty_like(W)
+            dist.broadcast(Wr, 0)
+    else:
+        W = dev_bf16(w.W)
+        Wr = dev_bf16(w.W_ref) if not fwd_only else None
     tokens = torch.from_numpy(w.tokens).to(dev)
     bp = libdpo.BatchArgs(H, W, tokens, w.prompt_len, w.completion_len, dtype="bf16")
     br = libdpo.BatchArgs(H, Wr, tokens, w.prompt_len, w.completion_len, dtype="bf16") if not fwd_only else None
@@ -354,6 +433,11 @@ def run_ours(args):
     h2d = H_host.numel() * 2 + tok_host.numel() * 4
     d2h = (w.R if fwd_only else 2 + 3 * B) * 4
 
+    # ------------------------------------------------------------ same-box cuBLAS reference
+    cublas = None
+    if not args.no_cublas_reference:
+        cublas = cublas_sustained(torch, dev, stream, seconds=1.5)
+
     # ------------------------------------------------------------ aggregate over ranks
     t = torch.tensor([ms, e2e_ms, float(Nc)], device=dev, dtype=torch.float64)
     if ws_n > 1:
@@ -405,7 +489,7 @@ def run_ours(args):
             "roofline": {"kernel": "k_tc_gemm<EpiLSE> (forward LM-head GEMM + online LSE)",
                          "bound": "tensor", "achieved": fwd_tflops, "peak": sustained,
                          "unit": "TFLOP/s", "frac": fwd_tflops / sustained,
-                         "traffic": None,
+                         "traffic": profiled_traffic(args.workload),
                          "algorithmic_per_launch": f"2*Nc*d*V = {gemm_flop:.4g} FLOP",
                          "peak_kind": f"bf16_tflops_sustained ({peak_src})"},
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
@@ -413,6 +497,7 @@ def run_ours(args):
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clk,
             "cpu_baseline": cpu,
+            "cublas_same_box": cublas,
             "peak_device_bytes": torch.cuda.max_memory_allocated(dev),
             "logits_fp32_bytes_avoided": 4 * Nc * w.V,
         }
@@ -431,6 +516,7 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(WL.CONFIGS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-cublas-reference", action="store_true")
     ap.add_argument("--cpu-tokens-per-row", type=int, default=64)
     ap.add_argument("--ref-tokens-per-row", type=int, default=4)
     args = ap.parse_args(argv)

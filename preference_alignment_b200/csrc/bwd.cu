@@ -160,21 +160,24 @@ cudaError_t launch_bwd_grad(const CUtensorMap& mapA, const CUtensorMap& mapB, in
                             const int* rowid, uint16_t* G, long long ldG, int grid,
                             const DevCtl& ctl, cudaStream_t st) {
   EpiGrad::Params p{y, lse, coef, rowid, G, ldG, Mc, V, tok0};
-  return launch_gemm<false, false, EpiGrad>(mapA, mapB, Mc, V, d, 0, p, grid, ctl, st);
+  return launch_gemm<false, false, EpiGrad>(mapA, mapB, Mc, V, d, 2, p, grid, ctl, st,
+                                            token_group(d));
 }
 
 cudaError_t launch_bwd_dh(const CUtensorMap& mapA, const CUtensorMap& mapB, int Mc, int V, int d,
                           int tok0, const int* dst, float* dH, int grid, const DevCtl& ctl,
                           cudaStream_t st) {
   EpiRows::Params p{dst, dH, Mc, d, tok0};
-  return launch_gemm<false, true, EpiRows>(mapA, mapB, Mc, d, V, 1, p, grid, ctl, st);
+  return launch_gemm<false, true, EpiRows>(mapA, mapB, Mc, d, V, DPO_GROUP_DH > 0 ? 3 : 1, p,
+                                           grid, ctl, st, DPO_GROUP_DH);
 }
 
 cudaError_t launch_bwd_dw(const CUtensorMap& mapA, const CUtensorMap& mapB, int Mc, int V, int d,
                           float* dW, int accumulate, int grid, const DevCtl& ctl,
                           cudaStream_t st) {
   EpiDW::Params p{dW, V, d, accumulate};
-  return launch_gemm<true, true, EpiDW>(mapA, mapB, V, d, Mc, 1, p, grid, ctl, st);
+  return launch_gemm<true, true, EpiDW>(mapA, mapB, V, d, Mc, DPO_GROUP_DW > 0 ? 3 : 1, p, grid,
+                                         ctl, st, DPO_GROUP_DW);
 }
 
 }  // namespace dpo

@@ -143,7 +143,8 @@ cudaError_t launch_fwd_lse(const CUtensorMap& mapA, const CUtensorMap& mapB, int
   EpiLSE::Params p{y, part, zy, Nc, V, ldp};
   // order 0: all token tiles of one vocab tile run together, so each W tile is
   // read from HBM once and served to the other CTAs from L2
-  return launch_gemm<false, false, EpiLSE>(mapA, mapB, Nc, V, d, 0, p, grid, ctl, st);
+  return launch_gemm<false, false, EpiLSE>(mapA, mapB, Nc, V, d, 2, p, grid, ctl, st,
+                                           token_group(d));
 }
 
 // ------------------------------------------------------------------ combine

@@ -7,6 +7,14 @@
 
 namespace dpo {
 
+// Token tiles (256 rows of packed H, K = d) per group of the forward raster: as
+// many as fit DPO_L2_GROUP_BYTES, at least one.
+inline int token_group(int d) {
+  const long long per_tile = 256ll * d * 2;
+  const long long g = DPO_L2_GROUP_BYTES / per_tile;
+  return g < 1 ? 1 : static_cast<int>(g);
+}
+
 // Clusters of two that can be resident at once for a pair-kernel instantiation
 // on the current device (cached per device).
 template <class Kern>
@@ -30,10 +38,13 @@ int max_pair_clusters(Kern kern, int smem_bytes) {
 
 // D[M x N] = A[M x K] . B[N x K]^T with the epilogue Epi; `order` picks the tile
 // raster (0: M fastest, 1: N fastest); `sms` is the device's SM count.
+// Raster: `order` as in GemmGeom (0, 1, or 2/3 grouped along M/N with `group`
+// 256-wide tiles per group; a group of 0 falls back to order 0).
 template <bool A_MN, bool B_MN, class Epi>
 cudaError_t launch_gemm(const CUtensorMap& mapA, const CUtensorMap& mapB, int M, int N, int K,
                         int order, const typename Epi::Params& p, int sms, const DevCtl& ctl,
-                        cudaStream_t st) {
+                        cudaStream_t st, int group = 0) {
+  if (order >= 2 && group <= 0) order = 0;
   const int n_tiles = (N + kBN - 1) / kBN;
   const int k_blocks = (K + kBK - 1) / kBK;
   {
@@ -43,7 +54,7 @@ cudaError_t launch_gemm(const CUtensorMap& mapA, const CUtensorMap& mapB, int M,
     if (e != cudaSuccess) return e;
     const int clusters = max_pair_clusters(kern, kPairSmemBytes);
     if (clusters > 0) {
-      GemmGeom g{(M + kPairM - 1) / kPairM, n_tiles, k_blocks, order};
+      GemmGeom g{(M + kPairM - 1) / kPairM, n_tiles, k_blocks, order, group > 0 ? group : 1};
       const int tiles = g.m_tiles * g.n_tiles;
       int pairs = clusters < sms / 2 ? clusters : sms / 2;
       if (pairs > tiles) pairs = tiles;
@@ -56,7 +67,8 @@ cudaError_t launch_gemm(const CUtensorMap& mapA, const CUtensorMap& mapB, int M,
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        kGemmSmemBytes);
   if (e != cudaSuccess) return e;
-  GemmGeom g{(M + kBM - 1) / kBM, n_tiles, k_blocks, order};
+  GemmGeom g{(M + kBM - 1) / kBM, n_tiles, k_blocks, order,
+             group > 0 ? (order == 2 ? 2 * group : group) : 1};
   const int tiles = g.m_tiles * g.n_tiles;
   kern<<<sms < tiles ? sms : tiles, kGemmThreads, kGemmSmemBytes, st>>>(mapA, mapB, g, p, ctl);
   return cudaGetLastError();

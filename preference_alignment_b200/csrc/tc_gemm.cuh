@@ -33,18 +33,41 @@ constexpr int kGemmSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*ba
 // Tile schedule: linear tile index -> (m tile, n tile).
 //   order 0: m fastest (all M tiles of one N tile run together: B tile shared via L2)
 //   order 1: n fastest (all N tiles of one M tile run together: A tile shared via L2)
+//   order 2: grouped along M: `group` consecutive M tiles are swept across every N
+//            tile (N outer, M inner) before the next group starts, so the group's
+//            A rows stay in L2 while B streams past them once per group
+//   order 3: grouped along N, the same with the roles of M and N exchanged
 struct GemmGeom {
   int m_tiles, n_tiles, k_blocks;
   int order;
+  int group;
 };
 
 __device__ __forceinline__ void tile_coords(const GemmGeom& g, int tile, int& mt, int& nt) {
   if (g.order == 0) {
     mt = tile % g.m_tiles;
     nt = tile / g.m_tiles;
-  } else {
+  } else if (g.order == 1) {
     mt = tile / g.n_tiles;
     nt = tile % g.n_tiles;
+  } else if (g.order == 2) {
+    const int per_group = g.group * g.n_tiles;
+    const int grp = tile / per_group;
+    const int first_m = grp * g.group;
+    const int rem = g.m_tiles - first_m;
+    const int gm = rem < g.group ? rem : g.group;
+    const int local = tile - grp * per_group;
+    nt = local / gm;
+    mt = first_m + local % gm;
+  } else {
+    const int per_group = g.group * g.m_tiles;
+    const int grp = tile / per_group;
+    const int first_n = grp * g.group;
+    const int rem = g.n_tiles - first_n;
+    const int gn = rem < g.group ? rem : g.group;
+    const int local = tile - grp * per_group;
+    mt = local / gn;
+    nt = first_n + local % gn;
   }
 }
 

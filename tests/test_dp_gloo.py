@@ -95,3 +95,12 @@ def test_bench_ranks_share_weights_and_not_batches():
     c = bench.rank_workload("small", 1)
     assert c.H.dtype == np.uint16
     assert np.all(b.prompt_len + b.completion_len <= b.L) and np.all(b.prompt_len >= 1)
+
+
+def test_rank_batch_without_weights_matches_full_draw():
+    import bench
+    full = bench.rank_workload("tiny", 1, weights=True)
+    light = bench.rank_workload("tiny", 1, weights=False)
+    assert light.W is None and light.W_ref is None
+    for k in ("prompt_len", "completion_len", "tokens", "H"):
+        assert np.array_equal(getattr(full, k), getattr(light, k))
