@@ -1,0 +1,137 @@
+"""Edge cases of the CUDA path against the oracle: extreme and ragged shapes,
+argument combinations, and replay of the whole step from a captured CUDA graph."""
+import numpy as np
+import pytest
+
+from oracle import dpo_oracle as O
+from preference_alignment_b200 import libdpo
+from preference_alignment_b200 import workloads as WL
+
+from dpo_harness import (DeviceWorkload, TOL_GRAD, TOL_LOSS, TOL_TOK, assert_seq_close, np64,
+                         rel_frob)
+
+pytestmark = pytest.mark.gpu
+
+
+def _fwd_bwd_check(w, coef_seed=0, bwd=True):
+    import torch
+    dw = DeviceWorkload(w)
+    H = WL.widen(w.H, w.dtype)
+    W = WL.widen(w.W, w.dtype)
+    o = O.seq_logprobs(H, W, w.tokens, w.prompt_len, w.completion_len)
+    seq, tok, lse = dw.forward(dw.W, want_grad=True)
+    assert libdpo.check() == libdpo.OK
+    assert np.abs(np64(tok) - o["tok_logp"]).max() <= TOL_TOK
+    assert_seq_close(np64(seq), o["seq_logp"])
+    if not bwd:
+        return
+    coef = np.random.default_rng(coef_seed).normal(0, 0.05, size=w.R).astype(np.float32)
+    dH, dW = dw.backward(lse, torch.from_numpy(coef).cuda())
+    assert libdpo.check() == libdpo.OK
+    oH, oW = O.backward(H, W, w.tokens, w.prompt_len, w.completion_len, coef.astype(np.float64))
+    assert rel_frob(np64(dH), oH) <= TOL_GRAD
+    assert rel_frob(np64(dW), oW) <= TOL_GRAD
+
+
+def test_more_rows_than_one_row_table_launch():
+    # R = 1100 > 1024 rows: the row table is uploaded by two launches
+    w = WL.make_custom(R=1100, L=10, d=64, V=300, dtype="bf16", seed=61, prompt_range=(1, 6))
+    _fwd_bwd_check(w)
+
+
+def test_vocab_not_a_multiple_of_8():
+    # the bf16 dz rows are padded to 1008 columns; the padding must never be read as data
+    w = WL.make_custom(R=4, L=200, d=128, V=1001, dtype="bf16", seed=62, prompt_range=(1, 80))
+    _fwd_bwd_check(w)
+
+
+def test_smallest_hidden_size():
+    w = WL.make_custom(R=4, L=60, d=8, V=500, dtype="bf16", seed=63, prompt_range=(1, 30))
+    _fwd_bwd_check(w)
+
+
+def test_large_vocab_small_hidden():
+    w = WL.make_custom(R=2, L=150, d=64, V=70001, dtype="bf16", seed=64, prompt_range=(1, 40))
+    _fwd_bwd_check(w)
+
+
+def test_scored_positions_exact_multiple_of_tile():
+    # Nc = 512 = two 256-row pair tiles, no ragged tail
+    w = WL.make_custom(R=4, L=200, d=64, V=300, dtype="bf16", seed=65, prompt_range=(1, 5))
+    w.prompt_len[:] = 40
+    w.completion_len[:] = 128
+    assert w.n_scored == 512
+    _fwd_bwd_check(w)
+
+
+def test_some_rows_empty():
+    w = WL.make_custom(R=6, L=120, d=64, V=400, dtype="bf16", seed=66, prompt_range=(1, 50))
+    w.completion_len[[1, 4]] = 0
+    _fwd_bwd_check(w)
+
+
+def test_backward_without_dH():
+    import torch
+    w = WL.make_custom(R=4, L=150, d=128, V=600, dtype="bf16", seed=67, prompt_range=(1, 50))
+    dw = DeviceWorkload(w)
+    _, _, lse = dw.forward(dw.W, want_grad=True)
+    coef = torch.linspace(-0.1, 0.1, 4, device="cuda")
+    _, dW1 = dw.backward(lse, coef)
+    _, dW2 = dw.backward(lse, coef, want_dH=False)
+    assert libdpo.check() == libdpo.OK
+    assert np.array_equal(np64(dW1), np64(dW2))
+
+
+def test_adjacent_layout_bf16_end_to_end():
+    w = WL.make_custom(R=8, L=160, d=256, V=900, dtype="bf16", seed=68, layout="adjacent",
+                       prompt_range=(1, 60), ref_std=0.05)
+    dw = DeviceWorkload(w)
+    H = WL.widen(w.H, "bf16")
+    op = O.seq_logprobs(H, WL.widen(w.W, "bf16"), w.tokens, w.prompt_len, w.completion_len)
+    orf = O.seq_logprobs(H, WL.widen(w.W_ref, "bf16"), w.tokens, w.prompt_len, w.completion_len)
+    ol = O.dpo_loss(op["seq_logp"], orf["seq_logp"], w.beta, "adjacent")
+    pol, _, _ = dw.forward(dw.W, want_grad=False)
+    ref, _, _ = dw.forward(dw.W_ref, want_grad=False)
+    out = dw.loss(pol, ref)
+    assert abs(out["loss"].item() - ol["loss"]) <= TOL_LOSS
+    np.testing.assert_allclose(np64(out["weights"]), ol["weights"], atol=1e-4)
+
+
+def test_whole_step_replays_from_a_cuda_graph():
+    """The four calls of a step are captured into one CUDA graph and replayed; the replay
+    gives the same outputs as the direct calls (all are deterministic)."""
+    import torch
+    w = WL.make_custom(R=8, L=300, d=256, V=1500, dtype="bf16", seed=69, prompt_range=(1, 100))
+    dw = DeviceWorkload(w)
+    bp, br = dw.batch(dw.W), dw.batch(dw.W_ref)
+    f, b, _ = libdpo.workspace_size(bp)
+    ws = torch.empty(max(f, b), dtype=torch.uint8, device="cuda")
+    R, B = w.R, w.R // 2
+    pol, ref = torch.empty(R, device="cuda"), torch.empty(R, device="cuda")
+    lse = torch.empty(w.n_scored, device="cuda")
+    outs = [torch.empty(n, device="cuda") for n in (1, 1, B, B, B, B, R)]
+    dH = torch.empty(R, w.L, w.d, device="cuda")
+    dW = torch.empty(w.V, w.d, device="cuda")
+
+    def step(stream):
+        libdpo.seq_logprobs(bp, True, pol, None, lse, ws, stream=stream)
+        libdpo.seq_logprobs(br, False, ref, None, None, ws, stream=stream)
+        libdpo.loss(B, w.layout, pol, ref, w.beta, 1.0, *outs, stream=stream)
+        libdpo.backward(bp, lse, outs[6], dH, dW, False, ws, stream=stream)
+
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        step(s.cuda_stream)                      # direct run (also sets up the kernels)
+    s.synchronize()
+    direct = [t.clone() for t in (pol, ref, lse, *outs, dH, dW)]
+    for t in (pol, ref, lse, *outs, dH, dW):
+        t.fill_(float("nan"))
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        step(s.cuda_stream)
+    g.replay()
+    g.replay()
+    torch.cuda.synchronize()
+    assert libdpo.check() == libdpo.OK
+    for a, b in zip(direct, (pol, ref, lse, *outs, dH, dW)):
+        assert torch.equal(a, b)
