@@ -148,11 +148,23 @@ def sigmoid(x):
     return e / (1.0 + e)
 
 
-def dpo_loss(pol, ref, beta, layout="halves", grad_scale=1.0):
+def dpo_loss(pol, ref, beta, layout="halves", grad_scale=1.0, completion_len=None,
+             normalize=False, nll_weight=0.0):
     """Sigmoid DPO loss and its metrics, from policy and reference sequence sums.
 
     pol, ref: [2B] sequence log-prob sums in the row layout. The log-ratios are
     formed first, then their difference, as the pages' dpo_step does.
+
+    Variants ("Run Distributed Full-Model DPO with PyTorch FSDP", Step 4: sums let
+    the loss use length-normalised or sum-based rewards; "DPO Training on GPU, in
+    depth", failure modes: length-normalised variants and an added SFT term; the
+    video transcript: total loss = DPO loss + lambda * NLL on the chosen responses):
+      normalize   use S_r / C_r (the average completion log-prob; 0 for C_r = 0)
+                  for policy and reference alike;
+      nll_weight  lambda: add lambda * NLL, the standard language-modelling loss on
+                  the chosen completions, read as the mean over all their tokens:
+                  NLL = -(sum of chosen S_r) / (sum of chosen C_r), from raw sums.
+    completion_len [2B] is needed by either variant.
     """
     pol = [float(x) for x in pol]
     ref = [float(x) for x in ref]
@@ -160,11 +172,19 @@ def dpo_loss(pol, ref, beta, layout="halves", grad_scale=1.0):
     if R % 2:
         raise ValueError("odd number of rows")
     B = R // 2
+    C = None if completion_len is None else [int(c) for c in completion_len]
+    if (normalize or nll_weight) and C is None:
+        raise ValueError("completion lengths are needed for the loss variants")
+    scale = [1.0] * R                      # d(value used in the loss)/d(raw sum)
+    if normalize:
+        scale = [1.0 / c if c > 0 else 0.0 for c in C]
+    pv = [pol[r] * scale[r] for r in range(R)]
+    rv = [ref[r] * scale[r] for r in range(R)]
     margins, rc, rr, w, losses = [], [], [], [], []
     coef = [0.0] * R
     for i, (c, r) in enumerate(pair_rows(B, layout)):
-        rho_c = pol[c] - ref[c]
-        rho_r = pol[r] - ref[r]
+        rho_c = pv[c] - rv[c]
+        rho_r = pv[r] - rv[r]
         m = beta * (rho_c - rho_r)
         margins.append(m)
         rc.append(beta * rho_c)
@@ -173,10 +193,20 @@ def dpo_loss(pol, ref, beta, layout="halves", grad_scale=1.0):
         w.append(wi)
         losses.append(softplus(-m))          # -log sigmoid(m)
         # d softplus(-m)/dm = -sigmoid(-m); dm/dpol[c] = beta, dm/dpol[r] = -beta
-        coef[c] = -grad_scale * beta * wi / B
-        coef[r] = +grad_scale * beta * wi / B
+        coef[c] = -grad_scale * beta * wi / B * scale[c]
+        coef[r] = +grad_scale * beta * wi / B * scale[r]
+    loss = math.fsum(losses) / B
+    nll = 0.0
+    if nll_weight:
+        chosen = [c for c, _ in pair_rows(B, layout)]
+        ntok = sum(C[c] for c in chosen)
+        if ntok > 0:
+            nll = -math.fsum(pol[c] for c in chosen) / ntok
+            for c in chosen:
+                coef[c] += -grad_scale * nll_weight / ntok
+        loss = loss + nll_weight * nll
     return {
-        "loss": math.fsum(losses) / B,
+        "loss": loss,
         "accuracy": sum(1.0 for m in margins if m > 0) / B,
         "margins": np.array(margins),
         "chosen_rewards": np.array(rc),
@@ -184,6 +214,7 @@ def dpo_loss(pol, ref, beta, layout="halves", grad_scale=1.0):
         "weights": np.array(w),
         "row_coef": np.array(coef),
         "losses": np.array(losses),
+        "nll": nll,
     }
 
 

@@ -305,3 +305,69 @@ def test_position_grad_h_matches_backward():
     for r, t in O.scored_positions(w.prompt_len, w.completion_len, w.L)[::3]:
         g = O.position_grad_h(H[r, t], W, w.tokens[r, t + 1], coef[r])
         np.testing.assert_allclose(g, dH[r, t], rtol=1e-12, atol=1e-14)
+
+
+# ---------------------------------------------------------------- loss variants
+def test_normalised_loss_with_unit_lengths_is_the_plain_loss():
+    rng = np.random.default_rng(31)
+    pol = -rng.uniform(1, 50, 8)
+    ref = pol + rng.normal(0, 2, 8)
+    a = O.dpo_loss(pol, ref, 0.1, "halves")
+    b = O.dpo_loss(pol, ref, 0.1, "halves", completion_len=np.ones(8, int), normalize=True)
+    assert a["loss"] == b["loss"]
+    np.testing.assert_array_equal(a["row_coef"], b["row_coef"])
+
+
+def test_normalised_loss_ignores_repeating_every_token():
+    # doubling every completion (C -> 2C, S -> 2S) leaves average log-probs, hence the loss,
+    # unchanged, while the plain sum-based loss changes
+    rng = np.random.default_rng(32)
+    C = rng.integers(1, 40, 8)
+    pol = -rng.uniform(0.5, 3, 8) * C
+    ref = pol + rng.normal(0, 1, 8)
+    a = O.dpo_loss(pol, ref, 0.2, "adjacent", completion_len=C, normalize=True)
+    b = O.dpo_loss(2 * pol, 2 * ref, 0.2, "adjacent", completion_len=2 * C, normalize=True)
+    assert b["loss"] == pytest.approx(a["loss"], rel=1e-14)
+    assert O.dpo_loss(2 * pol, 2 * ref, 0.2, "adjacent")["loss"] != pytest.approx(
+        O.dpo_loss(pol, ref, 0.2, "adjacent")["loss"], rel=1e-6)
+
+
+def test_nll_term_is_a_token_mean_over_chosen_completions():
+    # pair 0: chosen C = 1, S = -1; pair 1: chosen C = 3, S = -9. Token mean: 10 / 4 = 2.5
+    # (a per-pair mean of means would give 2.0). Policy == reference, so DPO gives ln 2.
+    pol = np.array([-1.0, -9.0, -5.0, -7.0])           # halves: chosen rows 0, 1
+    C = np.array([1, 3, 2, 2])
+    out = O.dpo_loss(pol, pol.copy(), 0.1, "halves", completion_len=C, nll_weight=0.5)
+    assert out["nll"] == 2.5
+    assert out["loss"] == pytest.approx(math.log(2) + 0.5 * 2.5, rel=1e-15)
+
+
+def test_nll_at_uniform_logits_is_log_vocab():
+    # W = 0: every chosen token has log p = -log V, so the NLL is log V whatever the lengths
+    w = WL.make_custom(R=6, L=40, d=8, V=53, dtype="f32", seed=33, prompt_range=(1, 20),
+                       min_completion=1)
+    H, W = _dense(w.H, w.W)
+    W[:] = 0.0
+    s = O.seq_logprobs(H, W, w.tokens, w.prompt_len, w.completion_len)["seq_logp"]
+    out = O.dpo_loss(s, s.copy(), 0.1, "halves", completion_len=w.completion_len, nll_weight=1.0)
+    assert out["nll"] == pytest.approx(math.log(53), rel=1e-13)
+
+
+@pytest.mark.parametrize("normalize,nll", [(True, 0.0), (False, 0.7), (True, 0.3)])
+def test_variant_row_coef_by_finite_differences(normalize, nll):
+    rng = np.random.default_rng(34)
+    B = 3
+    C = rng.integers(1, 30, 2 * B)
+    pol = -rng.uniform(0.5, 4, 2 * B) * C
+    ref = pol + rng.normal(0, 3, 2 * B)
+    for layout in ("halves", "adjacent"):
+        kw = dict(completion_len=C, normalize=normalize, nll_weight=nll)
+        out = O.dpo_loss(pol, ref, 0.1, layout, grad_scale=0.5, **kw)
+        eps = 1e-5
+        for r in range(2 * B):
+            p1, p2 = pol.copy(), pol.copy()
+            p1[r] += eps
+            p2[r] -= eps
+            fd = 0.5 * (O.dpo_loss(p1, ref, 0.1, layout, **kw)["loss"]
+                        - O.dpo_loss(p2, ref, 0.1, layout, **kw)["loss"]) / (2 * eps)
+            assert out["row_coef"][r] == pytest.approx(fd, rel=1e-6, abs=1e-12)
