@@ -132,6 +132,33 @@ dpo_status dpo_loss(int32_t B, int32_t layout, const float* pol, const float* re
                     float* chosen_rewards, float* rejected_rewards, float* weights,
                     float* row_coef, void* stream);
 
+/* Loss variants on the same per-row sums ("Run Distributed Full-Model DPO with
+ * PyTorch FSDP", Step 4: un-averaged sums let the loss use length-normalised or
+ * sum-based rewards; "DPO Training on GPU, in depth", failure modes: length-
+ * normalised variants and an added SFT term; the video transcript: total loss =
+ * DPO loss + lambda * a standard language-modelling NLL on the chosen responses).
+ *   normalize       1: the loss, rewards and margins use S_r / C_r (the average
+ *                   completion log-prob; 0 for C_r = 0) for policy and reference
+ *   nll_weight      lambda >= 0: add lambda * NLL, NLL = -(sum of the chosen rows'
+ *                   policy sums) / (their total completion length), i.e. the mean
+ *                   over all chosen completion tokens
+ *   completion_len  device [2B] int32 C_r in the row layout; required when
+ *                   normalize != 0 or nll_weight > 0, else may be NULL */
+typedef struct {
+  int32_t normalize;
+  float nll_weight;
+  const int32_t* completion_len;
+} dpo_loss_options;
+
+/* dpo_loss with the variants above (opt may be NULL: then it equals dpo_loss).
+ * row_coef stays d(grad_scale * loss)/d pol[row] and feeds dpo_backward as is.
+ *   nll   device [1] or NULL: the NLL value (0 when nll_weight is 0) */
+dpo_status dpo_loss_ex(int32_t B, int32_t layout, const float* pol, const float* ref, float beta,
+                       float grad_scale, const dpo_loss_options* opt, float* loss,
+                       float* accuracy, float* margins, float* chosen_rewards,
+                       float* rejected_rewards, float* weights, float* row_coef, float* nll,
+                       void* stream);
+
 /* Backward of sum_r row_coef[r] * seq_logp[r] (step 5) to H and W.
  *   lse_state   device [Nc] fp32 from dpo_seq_logprobs(want_grad=1) on the same batch
  *   row_coef    device [R] fp32, d(objective)/d seq_logp[r] (dpo_loss writes it)

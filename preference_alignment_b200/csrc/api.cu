@@ -277,9 +277,33 @@ dpo_status dpo_loss(int32_t B, int32_t layout, const float* pol, const float* re
   if (pol == nullptr || ref == nullptr || loss == nullptr) return DPO_ERR_INVALID_ARG;
   if (!(beta > 0.f) || !std::isfinite(beta) || !std::isfinite(grad_scale))
     return DPO_ERR_INVALID_ARG;
-  return cuda_status(launch_loss(B, layout, pol, ref, beta, grad_scale, loss, accuracy, margins,
-                                 chosen_rewards, rejected_rewards, weights, row_coef,
-                                 static_cast<cudaStream_t>(stream)));
+  return cuda_status(launch_loss(B, layout, pol, ref, beta, grad_scale, 0, 0.0, nullptr, loss,
+                                 accuracy, margins, chosen_rewards, rejected_rewards, weights,
+                                 row_coef, nullptr, static_cast<cudaStream_t>(stream)));
+}
+
+dpo_status dpo_loss_ex(int32_t B, int32_t layout, const float* pol, const float* ref, float beta,
+                       float grad_scale, const dpo_loss_options* opt, float* loss, float* accuracy,
+                       float* margins, float* chosen_rewards, float* rejected_rewards,
+                       float* weights, float* row_coef, float* nll, void* stream) {
+  if (B < 1 || B > (1 << 28) || (layout != DPO_PAIRS_HALVES && layout != DPO_PAIRS_ADJACENT))
+    return DPO_ERR_INVALID_ARG;
+  if (pol == nullptr || ref == nullptr || loss == nullptr) return DPO_ERR_INVALID_ARG;
+  if (!(beta > 0.f) || !std::isfinite(beta) || !std::isfinite(grad_scale))
+    return DPO_ERR_INVALID_ARG;
+  int normalize = 0;
+  float nll_weight = 0.f;
+  const int32_t* clen = nullptr;
+  if (opt != nullptr) {
+    normalize = opt->normalize ? 1 : 0;
+    nll_weight = opt->nll_weight;
+    clen = opt->completion_len;
+    if (!std::isfinite(nll_weight) || nll_weight < 0.f) return DPO_ERR_INVALID_ARG;
+    if ((normalize || nll_weight > 0.f) && clen == nullptr) return DPO_ERR_INVALID_ARG;
+  }
+  return cuda_status(launch_loss(B, layout, pol, ref, beta, grad_scale, normalize, nll_weight,
+                                 clen, loss, accuracy, margins, chosen_rewards, rejected_rewards,
+                                 weights, row_coef, nll, static_cast<cudaStream_t>(stream)));
 }
 
 dpo_status dpo_backward(const dpo_batch* batch, const float* lse_state, const float* row_coef,

@@ -75,9 +75,10 @@ cudaError_t launch_bwd_dw(const CUtensorMap& mapA, const CUtensorMap& mapB, int 
 
 // Loss kernel (fp64 inside).
 cudaError_t launch_loss(int B, int layout, const float* pol, const float* ref, double beta,
-                        double grad_scale, float* loss, float* accuracy, float* margins,
-                        float* chosen_rewards, float* rejected_rewards, float* weights,
-                        float* row_coef, cudaStream_t st);
+                        double grad_scale, int normalize, double nll_weight, const int* clen,
+                        float* loss, float* accuracy, float* margins, float* chosen_rewards,
+                        float* rejected_rewards, float* weights, float* row_coef, float* nll,
+                        cudaStream_t st);
 
 // fp32 SIMT path.
 cudaError_t launch_f32_fwd(const float* H, const float* W, const Sched& s, int Nc, int d, int V,

@@ -176,6 +176,29 @@ def loss(B: int, layout, pol, ref, beta: float, grad_scale: float, loss_out, acc
            "dpo_loss")
 
 
+class LossOptions(ctypes.Structure):
+    _fields_ = [("normalize", ctypes.c_int32), ("nll_weight", ctypes.c_float),
+                ("completion_len", ctypes.c_void_p)]
+
+
+def loss_ex(B: int, layout, pol, ref, beta: float, grad_scale: float, loss_out, accuracy=None,
+            margins=None, chosen_rewards=None, rejected_rewards=None, weights=None, row_coef=None,
+            nll=None, normalize=False, nll_weight=0.0, completion_len=None, stream=None):
+    """dpo_loss_ex: length-normalised and/or SFT-NLL variants (completion_len: device int32 [2B])."""
+    lib = load()
+    fn = lib.dpo_loss_ex
+    vp = ctypes.c_void_p
+    fn.argtypes = [ctypes.c_int32, ctypes.c_int32, vp, vp, ctypes.c_float, ctypes.c_float,
+                   ctypes.POINTER(LossOptions), vp, vp, vp, vp, vp, vp, vp, vp, vp]
+    fn.restype = ctypes.c_int
+    opt = LossOptions(1 if normalize else 0, float(nll_weight), _ptr(completion_len))
+    lay = LAYOUTS[layout] if isinstance(layout, str) else int(layout)
+    _check(fn(int(B), lay, _ptr(pol), _ptr(ref), float(beta), float(grad_scale), ctypes.byref(opt),
+              _ptr(loss_out), _ptr(accuracy), _ptr(margins), _ptr(chosen_rewards),
+              _ptr(rejected_rewards), _ptr(weights), _ptr(row_coef), _ptr(nll), _stream(stream)),
+           "dpo_loss_ex")
+
+
 def backward(batch: BatchArgs, lse_state, row_coef, dH, dW, accumulate_dW: bool, ws,
              ws_bytes=None, stream=None):
     _check(load().dpo_backward(ctypes.byref(batch.c), _ptr(lse_state), _ptr(row_coef), _ptr(dH),

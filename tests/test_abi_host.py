@@ -142,3 +142,12 @@ def test_noalloc_refuses_oversized_batches_on_the_host(lib):
 def test_wait_budget_roundtrip(lib):
     old = libdpo.set_wait_budget_ms(1234)
     assert libdpo.set_wait_budget_ms(old) == 1234
+
+
+@pytest.mark.parametrize("kw", [dict(normalize=True), dict(nll_weight=0.5),
+                                dict(nll_weight=-1.0, completion_len=FAKE),
+                                dict(nll_weight=float("nan"), completion_len=FAKE)])
+def test_loss_ex_rejects_bad_options(lib, kw):
+    with pytest.raises(libdpo.DpoError) as e:
+        libdpo.loss_ex(2, "halves", FAKE, FAKE, 0.1, 1.0, FAKE, **kw)
+    assert e.value.status == libdpo.ERR_INVALID_ARG
