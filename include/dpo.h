@@ -207,6 +207,16 @@ dpo_status dpo_check(void* stream);
  * (again bounded) and exit. Returns the previous value. */
 uint32_t dpo_set_wait_budget_ms(uint32_t ms);
 
+/* 64-bit fingerprint of a device buffer, for tagging offline reference scores with
+ * the weights they were computed from (Megatron-Bridge PR 6092: the scorer writes a
+ * metadata record next to the stored sums and the trainer refuses a mismatch).
+ *   data  device, 16-byte aligned, `bytes` long (bytes may be 0)
+ *   out   device [1] uint64, 8-byte aligned: written asynchronously on `stream`
+ * Each 16-byte word is hashed with its index through the splitmix64 finaliser
+ * (Steele, Lea and Flood, OOPSLA 2014) and the hashes are summed mod 2^64, so the
+ * value is the same for every launch configuration and run. Not cryptographic. */
+dpo_status dpo_fingerprint(const void* data, size_t bytes, uint64_t* out, void* stream);
+
 /* Self-test of the kernels' bounded waits: launches one CTA that waits, with the
  * same bounded wait the GEMM pipelines use, on a barrier nothing ever arrives on.
  * After budget_ms the wait gives up and records DPO_ERR_TIMEOUT in the status

@@ -393,6 +393,17 @@ dpo_status dpo_check(void* stream) {
   return static_cast<dpo_status>(v);
 }
 
+dpo_status dpo_fingerprint(const void* data, size_t bytes, uint64_t* out, void* stream) {
+  if (out == nullptr || reinterpret_cast<uintptr_t>(out) % 8 != 0) return DPO_ERR_INVALID_ARG;
+  if (bytes > 0 && (data == nullptr || reinterpret_cast<uintptr_t>(data) % 16 != 0))
+    return DPO_ERR_INVALID_ARG;
+  DevInfo di;
+  dpo_status s = device_info(&di);
+  if (s != DPO_OK) return s;
+  return cuda_status(launch_fingerprint(data, bytes, reinterpret_cast<unsigned long long*>(out),
+                                        di.sms, static_cast<cudaStream_t>(stream)));
+}
+
 dpo_status dpo_selftest_wait_timeout(uint32_t budget_ms, void* stream) {
   DevInfo di;
   dpo_status s = device_info(&di);

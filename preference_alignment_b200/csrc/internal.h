@@ -91,6 +91,10 @@ cudaError_t launch_f32_dh(const float* G, const float* W, const Sched& s, int to
 cudaError_t launch_f32_dw(const float* G, const float* H, const Sched& s, int tok0, int Mc, int d,
                           int V, float* dW, int accumulate, cudaStream_t st);
 
+// 64-bit order-independent fingerprint of a device buffer into out (device).
+cudaError_t launch_fingerprint(const void* data, unsigned long long bytes,
+                               unsigned long long* out, int sms, cudaStream_t st);
+
 // Bounded-wait self-test: one CTA waits on an mbarrier nothing arrives on.
 cudaError_t launch_wait_selftest(const DevCtl& ctl, cudaStream_t st);
 

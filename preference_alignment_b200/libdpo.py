@@ -215,6 +215,15 @@ def selftest_wait_timeout(budget_ms: int, stream=None):
     _check(fn(int(budget_ms), _stream(stream)), "dpo_selftest_wait_timeout")
 
 
+def fingerprint(data, nbytes, out, stream=None):
+    """dpo_fingerprint: 64-bit order-independent hash of a device buffer into out (device uint64)."""
+    lib = load()
+    fn = lib.dpo_fingerprint
+    fn.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_void_p]
+    fn.restype = ctypes.c_int
+    _check(fn(_ptr(data), int(nbytes), _ptr(out), _stream(stream)), "dpo_fingerprint")
+
+
 def check(stream=None) -> int:
     """Synchronise the stream and return (and clear) the device status word."""
     return load().dpo_check(_stream(stream))
