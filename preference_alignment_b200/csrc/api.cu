@@ -97,7 +97,8 @@ struct Plan {
   int Nc = 0;
   std::vector<int> row_start;          // [R + 1]
   // common prefix of both workspaces
-  size_t off_rs = 0, off_P = 0, off_y = 0, off_dst = 0, off_rowid = 0, off_hp = 0, prefix = 0;
+  size_t off_rs = 0, off_P = 0, off_y = 0, off_dst = 0, off_rowid = 0, off_sync = 0, off_hp = 0,
+         prefix = 0;
   // forward suffix
   int S = 0, ldp = 0;
   size_t off_part = 0, off_zy = 0, off_lp = 0, fwd_total = 0;
@@ -150,6 +151,7 @@ dpo_status make_plan(const dpo_batch* b, Plan* p) {
   p->off_y = take(sizeof(int) * Nc);
   p->off_dst = take(sizeof(int) * Nc);
   p->off_rowid = take(sizeof(int) * Nc);
+  p->off_sync = take(sizeof(int) * kSyncInts);
   p->off_hp = take(bf16 ? Nc * b->d * 2 : 0);
   p->prefix = o;
 
@@ -179,6 +181,7 @@ Sched sched_of(const Plan& p, void* ws) {
   s.y = reinterpret_cast<int*>(w + p.off_y);
   s.dst = reinterpret_cast<int*>(w + p.off_dst);
   s.rowid = reinterpret_cast<int*>(w + p.off_rowid);
+  s.sync = reinterpret_cast<int*>(w + p.off_sync);
   return s;
 }
 
@@ -253,8 +256,8 @@ dpo_status dpo_seq_logprobs(const dpo_batch* batch, int want_grad, float* seq_lo
       if (!make_map(&mA, w + p.off_hp, p.d, p.Nc, 2ull * p.d, kBK, kBoxRows) ||
           !make_map(&mB, batch->W, p.d, p.V, 2ull * p.d, kBK, kBoxRows))
         return DPO_ERR_CUDA;
-      if (launch_fwd_lse(mA, mB, p.Nc, p.V, p.d, sc.y, part, p.ldp, zy, di.sms, ctl, st) !=
-          cudaSuccess)
+      if (launch_fwd_lse(mA, mB, p.Nc, p.V, p.d, sc.y, part, p.ldp, zy, di.sms, sc.sync, ctl,
+                         st) != cudaSuccess)
         return DPO_ERR_CUDA;
     } else {
       if (launch_f32_fwd(static_cast<const float*>(batch->H), static_cast<const float*>(batch->W),
@@ -356,12 +359,14 @@ dpo_status dpo_backward(const dpo_batch* batch, const float* lse_state, const fl
           !make_map(&mHmn, hp0, p.d, mc, 2ull * p.d, kBoxMN, kBK))
         return DPO_ERR_CUDA;
       if (launch_bwd_grad(mHk, mWk, mc, p.V, p.d, tok0, sc.y, lse_state, row_coef, sc.rowid, G,
-                          p.ldG, di.sms, ctl, st) != cudaSuccess)
+                          p.ldG, di.sms, sc.sync, ctl, st) != cudaSuccess)
         return DPO_ERR_CUDA;
       if (dH != nullptr &&
-          launch_bwd_dh(mGk, mWmn, mc, p.V, p.d, tok0, sc.dst, dH, di.sms, ctl, st) != cudaSuccess)
+          launch_bwd_dh(mGk, mWmn, mc, p.V, p.d, tok0, sc.dst, dH, di.sms, sc.sync, ctl, st) !=
+              cudaSuccess)
         return DPO_ERR_CUDA;
-      if (launch_bwd_dw(mGmn, mHmn, mc, p.V, p.d, dW, acc, di.sms, ctl, st) != cudaSuccess)
+      if (launch_bwd_dw(mGmn, mHmn, mc, p.V, p.d, dW, acc, di.sms, sc.sync, ctl, st) !=
+          cudaSuccess)
         return DPO_ERR_CUDA;
     } else {
       float* G = reinterpret_cast<float*>(w + p.off_G);

@@ -138,13 +138,13 @@ struct EpiLSE {
 
 cudaError_t launch_fwd_lse(const CUtensorMap& mapA, const CUtensorMap& mapB, int Nc, int V,
                            int d, const int* y, float2* part, int ldp, float* zy, int grid,
-                           const DevCtl& ctl, cudaStream_t st) {
+                           int* sync, const DevCtl& ctl, cudaStream_t st) {
   if (Nc == 0) return cudaSuccess;
   EpiLSE::Params p{y, part, zy, Nc, V, ldp};
   // order 0: all token tiles of one vocab tile run together, so each W tile is
   // read from HBM once and served to the other CTAs from L2
   return launch_gemm<false, false, EpiLSE>(mapA, mapB, Nc, V, d, 2, p, grid, ctl, st,
-                                           token_group(d));
+                                           token_group(d), DPO_EPOCH_KB, sync, kSyncInts);
 }
 
 // ------------------------------------------------------------------ combine

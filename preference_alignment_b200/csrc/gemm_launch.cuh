@@ -43,7 +43,8 @@ int max_pair_clusters(Kern kern, int smem_bytes) {
 template <bool A_MN, bool B_MN, class Epi>
 cudaError_t launch_gemm(const CUtensorMap& mapA, const CUtensorMap& mapB, int M, int N, int K,
                         int order, const typename Epi::Params& p, int sms, const DevCtl& ctl,
-                        cudaStream_t st, int group = 0) {
+                        cudaStream_t st, int group = 0, int epoch = 0, int* sync = nullptr,
+                        int sync_len = 0) {
   if (order >= 2 && group <= 0) order = 0;
   const int n_tiles = (N + kBN - 1) / kBN;
   const int k_blocks = (K + kBK - 1) / kBK;
@@ -54,11 +55,22 @@ cudaError_t launch_gemm(const CUtensorMap& mapA, const CUtensorMap& mapB, int M,
     if (e != cudaSuccess) return e;
     const int clusters = max_pair_clusters(kern, kPairSmemBytes);
     if (clusters > 0) {
-      GemmGeom g{(M + kPairM - 1) / kPairM, n_tiles, k_blocks, order, group > 0 ? group : 1};
+      GemmGeom g{(M + kPairM - 1) / kPairM, n_tiles, k_blocks, order, group > 0 ? group : 1,
+                 0, nullptr};
       const int tiles = g.m_tiles * g.n_tiles;
       int pairs = clusters < sms / 2 ? clusters : sms / 2;
       if (pairs > tiles) pairs = tiles;
       if (pairs < 1) pairs = 1;
+      if (epoch > 0 && sync != nullptr) {
+        // epochs this launch can reach; pacing stays off if the counters do not fit
+        const long long per_pair = static_cast<long long>((tiles + pairs - 1) / pairs) * k_blocks;
+        if (per_pair / epoch + 1 < sync_len) {
+          e = cudaMemsetAsync(sync, 0, sizeof(int) * (per_pair / epoch + 2), st);
+          if (e != cudaSuccess) return e;
+          g.epoch = epoch;
+          g.sync = sync;
+        }
+      }
       kern<<<2 * pairs, kGemmThreads, kPairSmemBytes, st>>>(mapA, mapB, g, p, ctl);
       return cudaGetLastError();
     }
@@ -68,7 +80,7 @@ cudaError_t launch_gemm(const CUtensorMap& mapA, const CUtensorMap& mapB, int M,
                                        kGemmSmemBytes);
   if (e != cudaSuccess) return e;
   GemmGeom g{(M + kBM - 1) / kBM, n_tiles, k_blocks, order,
-             group > 0 ? (order == 2 ? 2 * group : group) : 1};
+             group > 0 ? (order == 2 ? 2 * group : group) : 1, 0, nullptr};
   const int tiles = g.m_tiles * g.n_tiles;
   kern<<<sms < tiles ? sms : tiles, kGemmThreads, kGemmSmemBytes, st>>>(mapA, mapB, g, p, ctl);
   return cudaGetLastError();

@@ -32,6 +32,7 @@ struct Sched {
   int* y;                 // [Nc] target token of each scored position (-1 = out of range)
   int* dst;               // [Nc] flat index r * L + t of each scored position
   int* rowid;             // [Nc] row of each scored position
+  int* sync;              // [kSyncInts] pacing counters of the GEMM launches
 };
 
 cudaError_t launch_upload_rows(const RowChunk& rc, int* row_start, int* prompt,
@@ -47,7 +48,7 @@ cudaError_t launch_prep(const uint16_t* H, const int* tokens, const Sched& s, in
 //   zy[i] = z at the target column (written by the tile that holds it)
 cudaError_t launch_fwd_lse(const CUtensorMap& mapA, const CUtensorMap& mapB, int Nc, int V,
                            int d, const int* y, float2* part, int ldp, float* zy, int grid,
-                           const DevCtl& ctl, cudaStream_t st);
+                           int* sync, const DevCtl& ctl, cudaStream_t st);
 
 // Combine the vocab-tile partials of each position into lse and lp = zy - lse.
 cudaError_t launch_combine(const float2* part, int ldp, int S, const float* zy, const int* y,
@@ -61,16 +62,16 @@ cudaError_t launch_rowsum(const float* lp, const int* row_start, const int* prom
 cudaError_t launch_bwd_grad(const CUtensorMap& mapA, const CUtensorMap& mapB, int Mc, int V,
                             int d, int tok0, const int* y, const float* lse, const float* coef,
                             const int* rowid, uint16_t* G, long long ldG, int grid,
-                            const DevCtl& ctl, cudaStream_t st);
+                            int* sync, const DevCtl& ctl, cudaStream_t st);
 
 // dH rows: out[dst[tok0 + i]] = (G . W)[i]   (A = G K-major, B = W MN-major)
 cudaError_t launch_bwd_dh(const CUtensorMap& mapA, const CUtensorMap& mapB, int Mc, int V, int d,
-                          int tok0, const int* dst, float* dH, int grid, const DevCtl& ctl,
-                          cudaStream_t st);
+                          int tok0, const int* dst, float* dH, int grid, int* sync,
+                          const DevCtl& ctl, cudaStream_t st);
 
 // dW (+)= G^T . Hp   (A = G MN-major, B = Hp MN-major)
 cudaError_t launch_bwd_dw(const CUtensorMap& mapA, const CUtensorMap& mapB, int Mc, int V, int d,
-                          float* dW, int accumulate, int grid, const DevCtl& ctl,
+                          float* dW, int accumulate, int grid, int* sync, const DevCtl& ctl,
                           cudaStream_t st);
 
 // Loss kernel (fp64 inside).

@@ -41,7 +41,33 @@ struct GemmGeom {
   int m_tiles, n_tiles, k_blocks;
   int order;
   int group;
+  // Optional pacing of the CTA pairs (0 = off): every `epoch` K blocks the leader
+  // producers meet at a counter in `sync` (sync[0] counts pairs that have finished,
+  // sync[1 + e] pairs past epoch e), so concurrent tiles stay within about one
+  // epoch of each other and keep sharing the operand lines in L2.
+  int epoch;
+  int* sync;
 };
+
+// A leader producer that has finished epoch e records it, then waits (bounded) until
+// every pair has finished epoch e - 1 (or has no work left). The one epoch of slack
+// keeps the fast pairs issuing loads while the slow ones catch up, and still bounds
+// the distance between any two pairs to about two epochs.
+__device__ __forceinline__ bool pace_epoch(const GemmGeom& g, int e, int n_pairs,
+                                           const DevCtl& ctl, volatile int* abort_flag) {
+  atomicAdd(g.sync + 1 + e, 1);
+  if (e == 0) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  while (true) {
+    int a, f;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(a) : "l"(g.sync + e) : "memory");
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(f) : "l"(g.sync) : "memory");
+    if (a + f >= n_pairs) return true;
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t0 > ctl.budget_ns) return false;
+    __nanosleep(64);
+  }
+}
 
 __device__ __forceinline__ void tile_coords(const GemmGeom& g, int tile, int& mt, int& nt) {
   if (g.order == 0) {
@@ -359,12 +385,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
+    long long gk = 0;                       // K blocks issued by this pair so far
+    const bool pacer = leader && g.epoch > 0;
     for (int tile = pair; tile < n_tiles_total && ok; tile += n_pairs) {
       int mt, nt;
       tile_coords(g, tile, mt, nt);
       const int arow = mt * kPairM + static_cast<int>(rank) * 128;
       const int brow = nt * kBN + static_cast<int>(rank) * (kBN / 2);
-      for (int kb = 0; kb < g.k_blocks; ++kb) {
+      for (int kb = 0; kb < g.k_blocks; ++kb, ++gk) {
+        if (pacer && gk > 0 && gk % g.epoch == 0 &&
+            !pace_epoch(g, static_cast<int>(gk / g.epoch) - 1, n_pairs, ctl, abort_flag)) {
+          ok = false;
+          break;
+        }
         if (!mbar_wait(empty0 + 8 * stage, phase ^ 1, ctl, abort_flag)) {
           ok = false;
           break;
@@ -391,6 +424,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         }
       }
     }
+    if (pacer) atomicAdd(g.sync, 1);        // finished: count as arrived at every later epoch
     if (!ok) {
       record_status(ctl, kStatusTimeout);
       *abort_flag = 1;
