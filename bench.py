@@ -88,7 +88,8 @@ class ClockSampler:
     def __init__(self, gpu_index):
         self.idx = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+        import tempfile
+        self.path = os.path.join(tempfile.gettempdir(), f"dpo_bench_clocks_{os.getpid()}_{gpu_index}.csv")
 
     def start(self):
         try:
@@ -296,6 +297,7 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
     libdpo.load()
+    libdpo.set_gemm_variant(args.gemm_variant)
 
     w = rank_workload(args.workload, rank, weights=(ws_n == 1 or rank == 0))
     B = w.R // 2
@@ -474,6 +476,7 @@ def run_ours(args):
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded; random-init LM-head weights of the Llama-3.1-8B head shape)",
             "config": {"workload": args.workload, "text": CONFIG_TEXT, "rows_per_gpu": w.R,
+                       "gemm_single_cta_mask": args.gemm_variant,
                        "pairs_per_gpu": B, "seq_len": w.L, "d": w.d, "V": w.V,
                        "scored_tokens_per_gpu": Nc, "global_batch_pairs": B * ws_n,
                        "parallelism": f"dp{ws_n}",
@@ -517,6 +520,8 @@ def main(argv=None):
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(WL.CONFIGS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-cublas-reference", action="store_true")
+    ap.add_argument("--gemm-variant", type=int, default=0, choices=range(16),
+                    help="mask, one bit per GEMM (forward, dz, dH, dW): set = single-CTA kernel")
     ap.add_argument("--cpu-tokens-per-row", type=int, default=64)
     ap.add_argument("--ref-tokens-per-row", type=int, default=4)
     args = ap.parse_args(argv)

@@ -25,6 +25,7 @@ constexpr size_t kAlign = 256;
 constexpr int kMinChunk = 128;   // smallest backward token chunk
 
 std::atomic<uint32_t> g_budget_ms{4000};
+std::atomic<int> g_gemm_variant{0};
 
 struct DevInfo {
   bool ready = false;
@@ -216,6 +217,8 @@ bool ws_ok(const void* ws, size_t have, size_t need) {
 }
 
 }  // namespace
+
+int dpo::gemm_variant() { return g_gemm_variant.load(); }
 
 extern "C" {
 
@@ -416,6 +419,11 @@ dpo_status dpo_selftest_wait_timeout(uint32_t budget_ms, void* stream) {
   DevCtl ctl = make_ctl(di);
   ctl.budget_ns = static_cast<unsigned long long>(budget_ms < 1 ? 1 : budget_ms) * 1000000ull;
   return cuda_status(launch_wait_selftest(ctl, static_cast<cudaStream_t>(stream)));
+}
+
+int32_t dpo_set_gemm_variant(int32_t variant) {
+  if (variant < 0 || variant > 15) return -1;
+  return g_gemm_variant.exchange(variant);
 }
 
 uint32_t dpo_set_wait_budget_ms(uint32_t ms) { return g_budget_ms.exchange(ms < 1 ? 1 : ms); }

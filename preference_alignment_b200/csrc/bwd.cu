@@ -161,7 +161,8 @@ cudaError_t launch_bwd_grad(const CUtensorMap& mapA, const CUtensorMap& mapB, in
                             int* sync, const DevCtl& ctl, cudaStream_t st) {
   EpiGrad::Params p{y, lse, coef, rowid, G, ldG, Mc, V, tok0};
   return launch_gemm<false, false, EpiGrad>(mapA, mapB, Mc, V, d, 2, p, grid, ctl, st,
-                                            token_group(d), DPO_EPOCH_KB, sync, kSyncInts);
+                                            kGemmGrad, token_group(d), DPO_EPOCH_KB, sync,
+                                            kSyncInts);
 }
 
 cudaError_t launch_bwd_dh(const CUtensorMap& mapA, const CUtensorMap& mapB, int Mc, int V, int d,
@@ -169,8 +170,8 @@ cudaError_t launch_bwd_dh(const CUtensorMap& mapA, const CUtensorMap& mapB, int 
                           const DevCtl& ctl, cudaStream_t st) {
   EpiRows::Params p{dst, dH, Mc, d, tok0};
   return launch_gemm<false, true, EpiRows>(mapA, mapB, Mc, d, V, DPO_GROUP_DH > 0 ? 3 : 1, p,
-                                           grid, ctl, st, DPO_GROUP_DH, DPO_EPOCH_KB, sync,
-                                           kSyncInts);
+                                           grid, ctl, st, kGemmDH, DPO_GROUP_DH, DPO_EPOCH_KB,
+                                           sync, kSyncInts);
 }
 
 cudaError_t launch_bwd_dw(const CUtensorMap& mapA, const CUtensorMap& mapB, int Mc, int V, int d,
@@ -178,7 +179,8 @@ cudaError_t launch_bwd_dw(const CUtensorMap& mapA, const CUtensorMap& mapB, int 
                           cudaStream_t st) {
   EpiDW::Params p{dW, V, d, accumulate};
   return launch_gemm<true, true, EpiDW>(mapA, mapB, V, d, Mc, DPO_GROUP_DW > 0 ? 3 : 1, p, grid,
-                                         ctl, st, DPO_GROUP_DW, DPO_EPOCH_KB, sync, kSyncInts);
+                                         ctl, st, kGemmDW, DPO_GROUP_DW, DPO_EPOCH_KB, sync,
+                                         kSyncInts);
 }
 
 }  // namespace dpo

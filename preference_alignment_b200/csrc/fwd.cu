@@ -144,7 +144,8 @@ cudaError_t launch_fwd_lse(const CUtensorMap& mapA, const CUtensorMap& mapB, int
   // order 0: all token tiles of one vocab tile run together, so each W tile is
   // read from HBM once and served to the other CTAs from L2
   return launch_gemm<false, false, EpiLSE>(mapA, mapB, Nc, V, d, 2, p, grid, ctl, st,
-                                           token_group(d), DPO_EPOCH_KB, sync, kSyncInts);
+                                           kGemmForward, token_group(d), DPO_EPOCH_KB, sync,
+                                           kSyncInts);
 }
 
 // ------------------------------------------------------------------ combine

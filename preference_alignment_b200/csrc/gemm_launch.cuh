@@ -3,6 +3,7 @@
 // is used when the device cannot co-schedule CTA pairs.
 #pragma once
 
+#include "internal.h"
 #include "tc_gemm.cuh"
 
 namespace dpo {
@@ -40,15 +41,16 @@ int max_pair_clusters(Kern kern, int smem_bytes) {
 // raster (0: M fastest, 1: N fastest); `sms` is the device's SM count.
 // Raster: `order` as in GemmGeom (0, 1, or 2/3 grouped along M/N with `group`
 // 256-wide tiles per group; a group of 0 falls back to order 0).
+// `kind` (a GemmKind) selects this GEMM's bit of the dpo_set_gemm_variant mask.
 template <bool A_MN, bool B_MN, class Epi>
 cudaError_t launch_gemm(const CUtensorMap& mapA, const CUtensorMap& mapB, int M, int N, int K,
                         int order, const typename Epi::Params& p, int sms, const DevCtl& ctl,
-                        cudaStream_t st, int group = 0, int epoch = 0, int* sync = nullptr,
-                        int sync_len = 0) {
+                        cudaStream_t st, int kind, int group = 0, int epoch = 0,
+                        int* sync = nullptr, int sync_len = 0) {
   if (order >= 2 && group <= 0) order = 0;
   const int n_tiles = (N + kBN - 1) / kBN;
   const int k_blocks = (K + kBK - 1) / kBK;
-  {
+  if (((gemm_variant() >> kind) & 1) == 0) {
     auto kern = k_tc_gemm_pair<A_MN, B_MN, Epi>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          kPairSmemBytes);

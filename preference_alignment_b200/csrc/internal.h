@@ -96,6 +96,12 @@ cudaError_t launch_f32_dw(const float* G, const float* H, const Sched& s, int to
 cudaError_t launch_fingerprint(const void* data, unsigned long long bytes,
                                unsigned long long* out, int sms, cudaStream_t st);
 
+// GEMM kernel selection, one bit per GEMM kind (dpo_set_gemm_variant): a set bit
+// runs that GEMM on the single-CTA kernel, a clear bit on CTA pairs when the device
+// can co-schedule them.
+enum GemmKind : int { kGemmForward = 0, kGemmGrad = 1, kGemmDH = 2, kGemmDW = 3 };
+int gemm_variant();
+
 // Bounded-wait self-test: one CTA waits on an mbarrier nothing arrives on.
 cudaError_t launch_wait_selftest(const DevCtl& ctl, cudaStream_t st);
 

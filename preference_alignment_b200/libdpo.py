@@ -224,6 +224,15 @@ def fingerprint(data, nbytes, out, stream=None):
     _check(fn(_ptr(data), int(nbytes), _ptr(out), _stream(stream)), "dpo_fingerprint")
 
 
+def set_gemm_variant(variant: int) -> int:
+    """Mask, one bit per GEMM (forward, dz, dH, dW): a set bit runs it on the single-CTA kernel."""
+    lib = load()
+    fn = lib.dpo_set_gemm_variant
+    fn.argtypes = [ctypes.c_int32]
+    fn.restype = ctypes.c_int32
+    return fn(int(variant))
+
+
 def check(stream=None) -> int:
     """Synchronise the stream and return (and clear) the device status word."""
     return load().dpo_check(_stream(stream))

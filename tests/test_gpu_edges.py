@@ -135,3 +135,35 @@ def test_whole_step_replays_from_a_cuda_graph():
     assert libdpo.check() == libdpo.OK
     for a, b in zip(direct, (pol, ref, lse, *outs, dH, dW)):
         assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("shape", [(6, 300, 256, 1000, 2), (8, 200, 200, 777, 3), (2, 700, 128, 2048, 4)])
+def test_single_cta_gemm_kernel(shape):
+    """The single-CTA GEMM (the fallback when CTA pairs cannot be co-scheduled) stays correct."""
+    R, L, d, V, seed = shape
+    w = WL.make_custom(R=R, L=L, d=d, V=V, dtype="bf16", seed=seed, prompt_range=(1, L // 3),
+                       full_rows=1)
+    old = libdpo.set_gemm_variant(15)
+    try:
+        _fwd_bwd_check(w)
+    finally:
+        libdpo.set_gemm_variant(old)
+
+
+def test_gemm_variants_agree():
+    import torch
+    w = WL.make_custom(R=4, L=400, d=256, V=1500, dtype="bf16", seed=91, prompt_range=(1, 100))
+    dw = DeviceWorkload(w)
+    outs = []
+    for v in (0, 15, 5):
+        old = libdpo.set_gemm_variant(v)
+        try:
+            seq, tok, lse = dw.forward(dw.W, want_grad=True)
+            dH, dW = dw.backward(lse, torch.linspace(-0.1, 0.1, 4, device="cuda"))
+        finally:
+            libdpo.set_gemm_variant(old)
+        outs.append((np64(tok), np64(dH), np64(dW)))
+    for o in outs[1:]:
+        assert np.abs(outs[0][0] - o[0]).max() <= 1e-4
+        assert rel_frob(outs[0][1], o[1]) <= 1e-3
+        assert rel_frob(outs[0][2], o[2]) <= 1e-3
