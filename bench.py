@@ -339,6 +339,9 @@ def run_ours(args):
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
 
     def step(timed=None):
+        step_with(bp, br, timed)
+
+    def step_with(bp, br, timed=None):
         if fwd_only:
             if timed is not None:
                 ev[0].record(stream)
@@ -409,26 +412,59 @@ def run_ours(args):
         raise RuntimeError(f"device status after timing: {libdpo.status_string(st)}")
 
     # ------------------------------------------------------------ end to end (host buffers)
+    # Every step uploads its inputs (H, tokens) from pinned host memory and reads its
+    # results (loss and metrics) back. As a training loop would, the upload of step
+    # i + 1 runs on a copy stream into the other of two input buffers while step i
+    # computes; the step waits for its own upload with an event.
     H_host = torch.from_numpy(np.ascontiguousarray(w.H).view(np.int16)).view(torch.bfloat16).pin_memory()
     tok_host = torch.from_numpy(w.tokens).pin_memory()
     res_host = torch.empty(max(2 + 3 * B, w.R), dtype=torch.float32).pin_memory()
     e2e_steps = max(3, min(args.steps, 20))
+    copy_stream = torch.cuda.Stream(dev)
+    H_buf = [H, torch.empty_like(H)]
+    tok_buf = [tokens, torch.empty_like(tokens)]
+    batches = []
+    for i in range(2):
+        if fwd_only:
+            batches.append((libdpo.BatchArgs(H_buf[i], W, tok_buf[i], w.prompt_len, w.completion_len,
+                                             dtype="bf16"), None))
+        else:
+            batches.append((libdpo.BatchArgs(H_buf[i], W, tok_buf[i], w.prompt_len, w.completion_len,
+                                             dtype="bf16"),
+                            libdpo.BatchArgs(H_buf[i], Wr, tok_buf[i], w.prompt_len, w.completion_len,
+                                             dtype="bf16")))
+    uploaded = [torch.cuda.Event() for _ in range(2)]
+    consumed = [torch.cuda.Event() for _ in range(2)]
+
+    def upload(i):
+        with torch.cuda.stream(copy_stream):
+            copy_stream.wait_event(consumed[i % 2])          # buffer free again
+            H_buf[i % 2].copy_(H_host, non_blocking=True)
+            tok_buf[i % 2].copy_(tok_host, non_blocking=True)
+            uploaded[i % 2].record(copy_stream)
+
+    for i in range(2):
+        consumed[i].record(stream)
     if ws_n > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(e2e_steps):
-        H.copy_(H_host, non_blocking=True)
-        tokens.copy_(tok_host, non_blocking=True)
-        step()
+    upload(0)
+    for i in range(e2e_steps):
+        if i + 1 < e2e_steps:
+            upload(i + 1)
+        stream.wait_event(uploaded[i % 2])
+        bp_i, br_i = batches[i % 2]
+        step_with(bp_i, br_i)
+        consumed[i % 2].record(stream)
         if fwd_only:
             res_dev = pol
         else:
             res_dev = torch.cat([outs["loss"], outs["accuracy"], outs["margins"], outs["cr"], outs["rr"]])
         res_host[:res_dev.numel()].copy_(res_dev, non_blocking=True)
-        stream.synchronize()
+        stream.synchronize()                                 # the host reads the step's result
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = e0.elapsed_time(e1)

@@ -330,6 +330,7 @@ dpo_status dpo_backward(const dpo_batch* batch, const float* lse_state, const fl
   // Token chunk that fits the workspace (a multiple of 128 unless it covers all).
   size_t rows_fit = (ws_bytes - p.off_G) / p.g_row_bytes;
   int Mc = static_cast<int>(std::min<size_t>(rows_fit, static_cast<size_t>(p.Nc)));
+  Mc = std::min(Mc, kMaxAccumK);           // dW's K: positions per chunk
   if (Mc < p.Nc) Mc = Mc / kMinChunk * kMinChunk;
   if (p.Nc > 0 && Mc < 1) return DPO_ERR_WORKSPACE;
 
@@ -364,10 +365,21 @@ dpo_status dpo_backward(const dpo_batch* batch, const float* lse_state, const fl
       if (launch_bwd_grad(mHk, mWk, mc, p.V, p.d, tok0, sc.y, lse_state, row_coef, sc.rowid, G,
                           p.ldG, di.sms, sc.sync, ctl, st) != cudaSuccess)
         return DPO_ERR_CUDA;
-      if (dH != nullptr &&
-          launch_bwd_dh(mGk, mWmn, mc, p.V, p.d, tok0, sc.dst, dH, di.sms, sc.sync, ctl, st) !=
-              cudaSuccess)
-        return DPO_ERR_CUDA;
+      // dH = dz . W reduces over the vocabulary: chunks of at most kMaxAccumK columns,
+      // the later ones added to the rows by the epilogue.
+      for (int v0 = 0; dH != nullptr && v0 < p.V; v0 += kMaxAccumK) {
+        const int vc = std::min(kMaxAccumK, p.V - v0);
+        CUtensorMap mGkc = mGk, mWmnc = mWmn;
+        if (v0 > 0 || vc < p.V) {
+          if (!make_map(&mGkc, G + v0, vc, mc, 2ull * p.ldG, kBK, kBoxRows) ||
+              !make_map(&mWmnc, static_cast<const uint16_t*>(batch->W) + static_cast<size_t>(v0) * p.d,
+                        p.d, vc, 2ull * p.d, kBoxMN, kBK))
+            return DPO_ERR_CUDA;
+        }
+        if (launch_bwd_dh(mGkc, mWmnc, mc, vc, p.d, tok0, sc.dst, dH, v0 > 0 ? 1 : 0, di.sms,
+                          sc.sync, ctl, st) != cudaSuccess)
+          return DPO_ERR_CUDA;
+      }
       if (launch_bwd_dw(mGmn, mHmn, mc, p.V, p.d, dW, acc, di.sms, sc.sync, ctl, st) !=
           cudaSuccess)
         return DPO_ERR_CUDA;

@@ -87,6 +87,7 @@ struct EpiRows {
     const int* dst;        // packed position -> flat row r * L + t
     float* out;            // dH [R * L, d]
     int Mc, d, tok0;
+    int accumulate;        // 1: add to the rows (later vocabulary chunks of K)
   };
   float* o;
   int nbase;
@@ -104,10 +105,19 @@ struct EpiRows {
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
       const int col = nbase + c * 32 + q * 4;
-      if (col < p.d)
-        *reinterpret_cast<float4*>(o + col) =
-            make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
-                        __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
+      if (col < p.d) {
+        float4 r = make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
+                               __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
+        float4* dst = reinterpret_cast<float4*>(o + col);
+        if (p.accumulate) {
+          const float4 old = *dst;
+          r.x += old.x;
+          r.y += old.y;
+          r.z += old.z;
+          r.w += old.w;
+        }
+        *dst = r;
+      }
     }
   }
 
@@ -166,9 +176,9 @@ cudaError_t launch_bwd_grad(const CUtensorMap& mapA, const CUtensorMap& mapB, in
 }
 
 cudaError_t launch_bwd_dh(const CUtensorMap& mapA, const CUtensorMap& mapB, int Mc, int V, int d,
-                          int tok0, const int* dst, float* dH, int grid, int* sync,
+                          int tok0, const int* dst, float* dH, int accumulate, int grid, int* sync,
                           const DevCtl& ctl, cudaStream_t st) {
-  EpiRows::Params p{dst, dH, Mc, d, tok0};
+  EpiRows::Params p{dst, dH, Mc, d, tok0, accumulate};
   return launch_gemm<false, true, EpiRows>(mapA, mapB, Mc, d, V, DPO_GROUP_DH > 0 ? 3 : 1, p,
                                            grid, ctl, st, kGemmDH, DPO_GROUP_DH, DPO_EPOCH_KB,
                                            sync, kSyncInts);

@@ -1,7 +1,9 @@
-// Exact-fp32 SIMT route for DPO_F32 inputs (small problems; no tensor cores).
-// Same quantities as the bf16 route: per scored position the log-sum-exp over
-// the full vocabulary and the target logit, then dz = coef * (onehot - softmax)
-// and its products with W and H. Each reduction runs in a fixed order.
+// SIMT route for DPO_F32 inputs (small problems; no tensor cores): fp32 inputs and
+// products, fp64 accumulation of the long reductions (over the vocabulary and over
+// the scored positions). Same quantities as the bf16 route: per scored position the
+// log-sum-exp over the full vocabulary and the target logit, then
+// dz = coef * (onehot - softmax) and its products with W and H. Each reduction runs
+// in a fixed order.
 #include <cmath>
 
 #include "internal.h"
@@ -27,19 +29,23 @@ __global__ void __launch_bounds__(256) k_f32_fwd(const float* __restrict__ H,
                                                  const float* __restrict__ W, Sched s, int d,
                                                  int V, float2* __restrict__ part,
                                                  float* __restrict__ zy) {
-  __shared__ float sm[8], ss[8];
+  __shared__ float sm[8];
+  __shared__ double ss[8];
   const int i = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const float* h = H + static_cast<long long>(s.dst[i]) * d;
   const int y = s.y[i];
-  float m = -INFINITY, sum = 0.f;
+  // running (max, sum of exp) in fp64: a vocabulary of millions of terms would
+  // swamp an fp32 running sum
+  float m = -INFINITY;
+  double sum = 0.0;
   for (int v = warp; v < V; v += 8) {
     const float z = warp_dot(h, W + static_cast<long long>(v) * d, d, lane);
     if (z > m) {
-      sum = sum * expf(m - z) + 1.f;
+      sum = sum * exp(static_cast<double>(m) - z) + 1.0;
       m = z;
     } else {
-      sum += expf(z - m);
+      sum += exp(static_cast<double>(z) - m);
     }
     if (v == y && lane == 0) zy[i] = z;
   }
@@ -49,17 +55,21 @@ __global__ void __launch_bounds__(256) k_f32_fwd(const float* __restrict__ H,
   }
   __syncthreads();
   if (threadIdx.x == 0) {
-    float M = -INFINITY, S = 0.f;
+    float M = -INFINITY;
+    double S = 0.0;
     for (int w = 0; w < 8; ++w) {
       if (sm[w] == -INFINITY) continue;            // warp saw no vocab row (V < 8)
       if (sm[w] > M) {
-        S = S * expf(M - sm[w]) + ss[w];
+        S = S * exp(static_cast<double>(M) - sm[w]) + ss[w];
         M = sm[w];
       } else {
-        S += ss[w] * expf(sm[w] - M);
+        S += ss[w] * exp(static_cast<double>(sm[w]) - M);
       }
     }
-    part[i] = make_float2(M, S);
+    // the combine stage takes (max, sum) in fp32; fold the sum's magnitude into the
+    // max so the fp32 value stays near 1 and loses nothing
+    const double ls = log(S);
+    part[i] = make_float2(static_cast<float>(M + ls), 1.f);
   }
 }
 
@@ -105,9 +115,10 @@ __global__ void __launch_bounds__(256) k_f32_dh(const float* __restrict__ G,
   const float* g = G + static_cast<long long>(i) * V;
   float* o = dH + static_cast<long long>(s.dst[tok0 + i]) * d;
   for (int k = threadIdx.x; k < d; k += blockDim.x) {
-    float a = 0.f;
-    for (int v = 0; v < V; ++v) a = fmaf(__ldg(g + v), __ldg(W + static_cast<long long>(v) * d + k), a);
-    o[k] = a;
+    double a = 0.0;     // fp64: V products per element
+    for (int v = 0; v < V; ++v)
+      a = fma(static_cast<double>(__ldg(g + v)), static_cast<double>(__ldg(W + static_cast<long long>(v) * d + k)), a);
+    o[k] = static_cast<float>(a);
   }
 }
 
@@ -126,11 +137,11 @@ __global__ void __launch_bounds__(256) k_f32_dw(const float* __restrict__ G,
   const int v = blockIdx.x;
   float* o = dW + static_cast<long long>(v) * d;
   for (int k = threadIdx.x; k < d; k += blockDim.x) {
-    float a = 0.f;
+    double a = 0.0;     // fp64: Mc products per element
     for (int i = 0; i < Mc; ++i)
-      a = fmaf(__ldg(G + static_cast<long long>(i) * V + v),
-               __ldg(H + static_cast<long long>(s.dst[tok0 + i]) * d + k), a);
-    o[k] = accumulate ? o[k] + a : a;
+      a = fma(static_cast<double>(__ldg(G + static_cast<long long>(i) * V + v)),
+              static_cast<double>(__ldg(H + static_cast<long long>(s.dst[tok0 + i]) * d + k)), a);
+    o[k] = accumulate ? o[k] + static_cast<float>(a) : static_cast<float>(a);
   }
 }
 

@@ -15,6 +15,13 @@ namespace dpo {
 
 constexpr int kRowChunk = 1024;   // rows uploaded per k_upload_rows launch (kernel parameter)
 
+// Longest reduction one tensor-core accumulator takes: the fp32 accumulation of a
+// tcgen05 MMA chain rounds with a small bias per step, which grows linearly with K
+// (measured: ~2% of dH at K = 2^24, negligible at 2^17). Longer reductions (dH over
+// a vocabulary beyond it, dW over more scored positions) are split into chunks
+// added together in fp32 by the epilogue.
+constexpr int kMaxAccumK = 1 << 20;
+
 // Row table slice passed by value to k_upload_rows.
 struct RowChunk {
   int row0;                       // first row of the slice
@@ -66,7 +73,7 @@ cudaError_t launch_bwd_grad(const CUtensorMap& mapA, const CUtensorMap& mapB, in
 
 // dH rows: out[dst[tok0 + i]] = (G . W)[i]   (A = G K-major, B = W MN-major)
 cudaError_t launch_bwd_dh(const CUtensorMap& mapA, const CUtensorMap& mapB, int Mc, int V, int d,
-                          int tok0, const int* dst, float* dH, int grid, int* sync,
+                          int tok0, const int* dst, float* dH, int accumulate, int grid, int* sync,
                           const DevCtl& ctl, cudaStream_t st);
 
 // dW (+)= G^T . Hp   (A = G MN-major, B = Hp MN-major)

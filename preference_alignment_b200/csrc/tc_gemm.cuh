@@ -1,5 +1,6 @@
-// Persistent, warp-specialised bf16 GEMM on the 5th-generation tensor cores
-// (tcgen05.mma, cta_group::1) with a pluggable per-row epilogue.
+// Persistent, warp-specialised bf16 GEMMs on the 5th-generation tensor cores with a
+// pluggable per-row epilogue: k_tc_gemm (one CTA per tile, tcgen05.mma cta_group::1)
+// and k_tc_gemm_pair (two CTAs of a cluster per tile, cta_group::2; the default).
 //
 //   D[M x N] = A[M x K] . B[N x K]^T     (fp32 accumulation in tensor memory)
 //
@@ -8,7 +9,8 @@
 // contiguous) or MN-major (rows of M or N contiguous, i.e. the transposed
 // storage); the shared-memory descriptor and the TMA boxes follow.
 //
-// Roles (192 threads, one CTA per SM, persistent over a static tile schedule):
+// Roles of the single-CTA kernel (192 threads, one CTA per SM, persistent over a
+// static tile schedule; the pair kernel below splits them across the pair):
 //   warp 0     one thread issues the TMA loads,
 //   warp 1     allocates 512 TMEM columns; one thread issues the MMAs,
 //   warps 2-5  epilogue: each thread owns one accumulator row (TMEM lane) and
@@ -43,8 +45,8 @@ struct GemmGeom {
   int group;
   // Optional pacing of the CTA pairs (0 = off): every `epoch` K blocks the leader
   // producers meet at a counter in `sync` (sync[0] counts pairs that have finished,
-  // sync[1 + e] pairs past epoch e), so concurrent tiles stay within about one
-  // epoch of each other and keep sharing the operand lines in L2.
+  // sync[1 + e] pairs past epoch e), so concurrent tiles stay within about two
+  // epochs of each other and keep sharing the operand lines in L2.
   int epoch;
   int* sync;
 };

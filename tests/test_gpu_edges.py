@@ -167,3 +167,14 @@ def test_gemm_variants_agree():
         assert np.abs(outs[0][0] - o[0]).max() <= 1e-4
         assert rel_frob(outs[0][1], o[1]) <= 1e-3
         assert rel_frob(outs[0][2], o[2]) <= 1e-3
+
+
+@pytest.mark.parametrize("R,L,d,V,seed", [
+    (2, 8, 8, 1 << 24, 101),      # the largest vocabulary the boundary accepts (65,536 vocab tiles)
+    (2, 8, 65536, 64, 102),       # the largest hidden size (1,024 K blocks per tile)
+    (65535, 2, 8, 16, 103),       # the most rows (64 row-table launches, one position each)
+])
+def test_maximum_sizes(R, L, d, V, seed):
+    w = WL.make_custom(R=R, L=L, d=d, V=V, dtype="bf16", seed=seed, prompt_range=(1, 1),
+                       min_completion=1)
+    _fwd_bwd_check(w)
