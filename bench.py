@@ -525,7 +525,7 @@ def run_ours(args):
             "batch_tokens_per_s": w.R * w.L * ws_n * args.steps / (ms / 1e3),
             "breakdown_ms": {"policy_fwd": float(bd[0]), "ref_fwd": float(bd[1]),
                              "loss": float(bd[2]), "backward": float(bd[3])},
-            "roofline": {"kernel": "k_tc_gemm<EpiLSE> (forward LM-head GEMM + online LSE)",
+            "roofline": {"kernel": "k_tc_gemm_pair<EpiLSE> (forward LM-head GEMM + online LSE)",
                          "bound": "tensor", "achieved": fwd_tflops, "peak": sustained,
                          "unit": "TFLOP/s", "frac": fwd_tflops / sustained,
                          "traffic": profiled_traffic(args.workload),

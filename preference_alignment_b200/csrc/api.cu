@@ -75,9 +75,10 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 2-D bf16 tensor map over a row-major [outer, inner] array with 128-byte swizzle.
+// 2-D bf16 tensor map over a row-major [outer, inner] array with 128-byte swizzle
+// (or none, for the epilogue's 32 x 32 store boxes).
 bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
-              uint32_t box_inner, uint32_t box_outer) {
+              uint32_t box_inner, uint32_t box_outer, bool swizzle = true) {
   auto fn = encode_fn();
   if (fn == nullptr) return false;
   cuuint64_t dims[2] = {inner, outer};
@@ -86,7 +87,8 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, 
   cuuint32_t es[2] = {1, 1};
   const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
                         strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -354,16 +356,17 @@ dpo_status dpo_backward(const dpo_batch* batch, const float* lse_state, const fl
     if (bf16) {
       uint16_t* G = reinterpret_cast<uint16_t*>(w + p.off_G);
       const uint16_t* hp0 = Hp + static_cast<size_t>(tok0) * p.d;
-      CUtensorMap mHk, mWk, mGk, mWmn, mGmn, mHmn;
-      if (!make_map(&mHk, hp0, p.d, mc, 2ull * p.d, kBK, kBoxRows) ||
+      CUtensorMap mHk, mWk, mGk, mWmn, mGmn, mHmn, mGst;
+      if (!make_map(&mGst, G, p.V, mc, 2ull * p.ldG, 32, 32, false) ||
+          !make_map(&mHk, hp0, p.d, mc, 2ull * p.d, kBK, kBoxRows) ||
           !make_map(&mWk, batch->W, p.d, p.V, 2ull * p.d, kBK, kBoxRows) ||
           !make_map(&mGk, G, p.V, mc, 2ull * p.ldG, kBK, kBoxRows) ||
           !make_map(&mWmn, batch->W, p.d, p.V, 2ull * p.d, kBoxMN, kBK) ||
           !make_map(&mGmn, G, p.V, mc, 2ull * p.ldG, kBoxMN, kBK) ||
           !make_map(&mHmn, hp0, p.d, mc, 2ull * p.d, kBoxMN, kBK))
         return DPO_ERR_CUDA;
-      if (launch_bwd_grad(mHk, mWk, mc, p.V, p.d, tok0, sc.y, lse_state, row_coef, sc.rowid, G,
-                          p.ldG, di.sms, sc.sync, ctl, st) != cudaSuccess)
+      if (launch_bwd_grad(mHk, mWk, mGst, mc, p.V, p.d, tok0, sc.y, lse_state, row_coef,
+                          sc.rowid, di.sms, sc.sync, ctl, st) != cudaSuccess)
         return DPO_ERR_CUDA;
       // dH = dz . W reduces over the vocabulary: chunks of at most kMaxAccumK columns,
       // the later ones added to the rows by the epilogue.

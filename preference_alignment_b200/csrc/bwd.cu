@@ -23,58 +23,66 @@ namespace dpo {
 constexpr float kLog2eB = 1.4426950408889634f;
 
 // ------------------------------------------------------------------ dz epilogue
+// Each thread forms its row's 32 bf16 values of a chunk; the warp stages its 32 x 32
+// block in shared memory and one lane stores it with a TMA bulk tensor store (rows
+// beyond the chunk and columns beyond V fall outside the tensor map and are skipped).
+// Two staging buffers per warp: a buffer is refilled only after the store issued
+// from it two chunks earlier has finished reading it.
 struct EpiGrad {
   struct Params {
     const int* y;
     const float* lse;
     const float* coef;     // [R] per-row coefficient
     const int* rowid;
-    uint16_t* G;           // [Mc, ldG] bf16 chunk
-    long long ldG;
     int Mc, V, tok0;
   };
-  int vbase, yl;
-  bool valid;
+  int vbase, yl, row0;
   float nl2, cf;
-  uint16_t* out;
+  EpiCtx ctx;
 
-  __device__ __forceinline__ void begin(const Params& p, int m_row, int nt) {
+  __device__ __forceinline__ void begin(const Params& p, int m_row, int nt, const EpiCtx& c) {
     const int tok = m_row;
-    valid = tok < p.Mc;
+    ctx = c;
+    row0 = tok - c.lane;                 // first row of this warp's 32-row block
     vbase = nt * kBN;
     yl = -1;
     nl2 = 0.f;
-    cf = 0.f;
-    out = nullptr;
-    if (valid) {
+    cf = 0.f;                            // rows past the chunk compute zeros (not stored)
+    if (tok < p.Mc) {
       const int gt = p.tok0 + tok;
       const int y = __ldg(p.y + gt);
       yl = y - vbase;
       nl2 = -__ldg(p.lse + gt) * kLog2eB;
       cf = y >= 0 ? __ldg(p.coef + __ldg(p.rowid + gt)) : 0.f;  // bad target: no gradient
-      out = p.G + static_cast<long long>(tok) * p.ldG + vbase;
     }
   }
 
-  __device__ __forceinline__ void chunk(const Params& p, int c, const uint32_t (&v)[32]) {
-    if (!valid) return;
+  __device__ __forceinline__ void chunk(const Params&, int c, const uint32_t (&v)[32]) {
     uint32_t packed[16];
 #pragma unroll
     for (int j = 0; j < 32; j += 2) {
       const int col = c * 32 + j;
-      float g0 = cf * ((col == yl ? 1.f : 0.f) -
-                       ex2_approx(fmaf(__uint_as_float(v[j]), kLog2eB, nl2)));
-      float g1 = cf * ((col + 1 == yl ? 1.f : 0.f) -
-                       ex2_approx(fmaf(__uint_as_float(v[j + 1]), kLog2eB, nl2)));
-      if (vbase + col >= p.V) g0 = 0.f;
-      if (vbase + col + 1 >= p.V) g1 = 0.f;
+      const float g0 = cf * ((col == yl ? 1.f : 0.f) -
+                             ex2_approx(fmaf(__uint_as_float(v[j]), kLog2eB, nl2)));
+      const float g1 = cf * ((col + 1 == yl ? 1.f : 0.f) -
+                             ex2_approx(fmaf(__uint_as_float(v[j + 1]), kLog2eB, nl2)));
       packed[j / 2] = pack_bf16x2(g0, g1);
     }
-    uint4* dst = reinterpret_cast<uint4*>(out + c * 32);
+    const uint32_t buf = ctx.stage + (c & 1) * (kEpiWarpBytes / 2);
+    if (ctx.lane == 0) bulk_wait_group_read<1>();   // the store from this buffer is done
+    __syncwarp();
+    const uint32_t dst = buf + ctx.lane * 64;       // row `lane`: 32 bf16 = 64 bytes
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      if (vbase + c * 32 + q * 8 < p.ldG)
-        dst[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+    for (int q = 0; q < 4; ++q)
+      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst + 16 * q),
+                   "r"(packed[4 * q]), "r"(packed[4 * q + 1]), "r"(packed[4 * q + 2]),
+                   "r"(packed[4 * q + 3])
+                   : "memory");
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (ctx.lane == 0 && row0 >= 0) {
+      tma_store_2d(ctx.map, buf, vbase + c * 32, row0);
+      bulk_commit_group();
     }
   }
 
@@ -93,7 +101,7 @@ struct EpiRows {
   int nbase;
   bool valid;
 
-  __device__ __forceinline__ void begin(const Params& p, int m_row, int nt) {
+  __device__ __forceinline__ void begin(const Params& p, int m_row, int nt, const EpiCtx&) {
     const int tok = m_row;
     valid = tok < p.Mc;
     nbase = nt * kBN;
@@ -134,7 +142,7 @@ struct EpiDW {
   int nbase;
   bool valid;
 
-  __device__ __forceinline__ void begin(const Params& p, int m_row, int nt) {
+  __device__ __forceinline__ void begin(const Params& p, int m_row, int nt, const EpiCtx&) {
     const int v = m_row;
     valid = v < p.V;
     nbase = nt * kBN;
@@ -165,12 +173,12 @@ struct EpiDW {
   __device__ __forceinline__ void end(const Params&) {}
 };
 
-cudaError_t launch_bwd_grad(const CUtensorMap& mapA, const CUtensorMap& mapB, int Mc, int V,
-                            int d, int tok0, const int* y, const float* lse, const float* coef,
-                            const int* rowid, uint16_t* G, long long ldG, int grid,
+cudaError_t launch_bwd_grad(const CUtensorMap& mapA, const CUtensorMap& mapB,
+                            const CUtensorMap& mapG, int Mc, int V, int d, int tok0, const int* y,
+                            const float* lse, const float* coef, const int* rowid, int grid,
                             int* sync, const DevCtl& ctl, cudaStream_t st) {
-  EpiGrad::Params p{y, lse, coef, rowid, G, ldG, Mc, V, tok0};
-  return launch_gemm<false, false, EpiGrad>(mapA, mapB, Mc, V, d, 2, p, grid, ctl, st,
+  EpiGrad::Params p{y, lse, coef, rowid, Mc, V, tok0};
+  return launch_gemm<false, false, EpiGrad>(mapA, mapB, mapG, Mc, V, d, 2, p, grid, ctl, st,
                                             kGemmGrad, token_group(d), DPO_EPOCH_KB, sync,
                                             kSyncInts);
 }
@@ -179,7 +187,7 @@ cudaError_t launch_bwd_dh(const CUtensorMap& mapA, const CUtensorMap& mapB, int 
                           int tok0, const int* dst, float* dH, int accumulate, int grid, int* sync,
                           const DevCtl& ctl, cudaStream_t st) {
   EpiRows::Params p{dst, dH, Mc, d, tok0, accumulate};
-  return launch_gemm<false, true, EpiRows>(mapA, mapB, Mc, d, V, DPO_GROUP_DH > 0 ? 3 : 1, p,
+  return launch_gemm<false, true, EpiRows>(mapA, mapB, mapA, Mc, d, V, DPO_GROUP_DH > 0 ? 3 : 1, p,
                                            grid, ctl, st, kGemmDH, DPO_GROUP_DH, DPO_EPOCH_KB,
                                            sync, kSyncInts);
 }
@@ -188,7 +196,7 @@ cudaError_t launch_bwd_dw(const CUtensorMap& mapA, const CUtensorMap& mapB, int 
                           float* dW, int accumulate, int grid, int* sync, const DevCtl& ctl,
                           cudaStream_t st) {
   EpiDW::Params p{dW, V, d, accumulate};
-  return launch_gemm<true, true, EpiDW>(mapA, mapB, V, d, Mc, DPO_GROUP_DW > 0 ? 3 : 1, p, grid,
+  return launch_gemm<true, true, EpiDW>(mapA, mapB, mapA, V, d, Mc, DPO_GROUP_DW > 0 ? 3 : 1, p, grid,
                                          ctl, st, kGemmDW, DPO_GROUP_DW, DPO_EPOCH_KB, sync,
                                          kSyncInts);
 }

@@ -42,11 +42,13 @@ int max_pair_clusters(Kern kern, int smem_bytes) {
 // Raster: `order` as in GemmGeom (0, 1, or 2/3 grouped along M/N with `group`
 // 256-wide tiles per group; a group of 0 falls back to order 0).
 // `kind` (a GemmKind) selects this GEMM's bit of the dpo_set_gemm_variant mask.
+// mapC is the epilogue's store tensor map (epilogues that do not store through TMA
+// ignore it; pass any valid map).
 template <bool A_MN, bool B_MN, class Epi>
-cudaError_t launch_gemm(const CUtensorMap& mapA, const CUtensorMap& mapB, int M, int N, int K,
-                        int order, const typename Epi::Params& p, int sms, const DevCtl& ctl,
-                        cudaStream_t st, int kind, int group = 0, int epoch = 0,
-                        int* sync = nullptr, int sync_len = 0) {
+cudaError_t launch_gemm(const CUtensorMap& mapA, const CUtensorMap& mapB, const CUtensorMap& mapC,
+                        int M, int N, int K, int order, const typename Epi::Params& p, int sms,
+                        const DevCtl& ctl, cudaStream_t st, int kind, int group = 0,
+                        int epoch = 0, int* sync = nullptr, int sync_len = 0) {
   if (order >= 2 && group <= 0) order = 0;
   const int n_tiles = (N + kBN - 1) / kBN;
   const int k_blocks = (K + kBK - 1) / kBK;
@@ -73,7 +75,7 @@ cudaError_t launch_gemm(const CUtensorMap& mapA, const CUtensorMap& mapB, int M,
           g.sync = sync;
         }
       }
-      kern<<<2 * pairs, kGemmThreads, kPairSmemBytes, st>>>(mapA, mapB, g, p, ctl);
+      kern<<<2 * pairs, kGemmThreads, kPairSmemBytes, st>>>(mapA, mapB, mapC, g, p, ctl);
       return cudaGetLastError();
     }
   }
@@ -84,7 +86,8 @@ cudaError_t launch_gemm(const CUtensorMap& mapA, const CUtensorMap& mapB, int M,
   GemmGeom g{(M + kBM - 1) / kBM, n_tiles, k_blocks, order,
              group > 0 ? (order == 2 ? 2 * group : group) : 1, 0, nullptr};
   const int tiles = g.m_tiles * g.n_tiles;
-  kern<<<sms < tiles ? sms : tiles, kGemmThreads, kGemmSmemBytes, st>>>(mapA, mapB, g, p, ctl);
+  kern<<<sms < tiles ? sms : tiles, kGemmThreads, kGemmSmemBytes, st>>>(mapA, mapB, mapC, g, p,
+                                                                        ctl);
   return cudaGetLastError();
 }
 

@@ -65,10 +65,11 @@ cudaError_t launch_combine(const float2* part, int ldp, int S, const float* zy, 
 cudaError_t launch_rowsum(const float* lp, const int* row_start, const int* prompt, int R, int L,
                           float* seq, float* tok_logp, cudaStream_t st);
 
-// Backward (bf16): G = coef * (onehot - softmax) for packed positions [tok0, tok0 + Mc).
-cudaError_t launch_bwd_grad(const CUtensorMap& mapA, const CUtensorMap& mapB, int Mc, int V,
-                            int d, int tok0, const int* y, const float* lse, const float* coef,
-                            const int* rowid, uint16_t* G, long long ldG, int grid,
+// Backward (bf16): G = coef * (onehot - softmax) for packed positions [tok0, tok0 + Mc),
+// stored through mapG (a [Mc, V] bf16 view of the dz chunk, 32 x 32 boxes, no swizzle).
+cudaError_t launch_bwd_grad(const CUtensorMap& mapA, const CUtensorMap& mapB,
+                            const CUtensorMap& mapG, int Mc, int V, int d, int tok0, const int* y,
+                            const float* lse, const float* coef, const int* rowid, int grid,
                             int* sync, const DevCtl& ctl, cudaStream_t st);
 
 // dH rows: out[dst[tok0 + i]] = (G . W)[i]   (A = G K-major, B = W MN-major)

@@ -30,7 +30,19 @@ constexpr int kBBytes = kBN * kBK * 2;   // 32 KiB
 constexpr int kStageBytes = kABytes + kBBytes;
 constexpr int kGemmThreads = 192;
 constexpr int kTmemCols = 512;
-constexpr int kGemmSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+// Per epilogue warp: two 32 x 32 bf16 staging buffers for TMA stores.
+constexpr int kEpiWarpBytes = 2 * 32 * 32 * 2;
+constexpr int kEpiSmemBytes = 4 * kEpiWarpBytes;      // 16 KiB
+constexpr int kGemmSmemBytes =
+    kStages * kStageBytes + kEpiSmemBytes + 1024 /*align*/ + 256 /*barriers*/;
+
+// What an epilogue thread may use besides its accumulator row: the store tensor
+// map and its warp's shared-memory staging buffers.
+struct EpiCtx {
+  const CUtensorMap* map;
+  uint32_t stage;     // shared address of this warp's kEpiWarpBytes
+  int lane;
+};
 
 // Tile schedule: linear tile index -> (m tile, n tile).
 //   order 0: m fastest (all M tiles of one N tile run together: B tile shared via L2)
@@ -99,20 +111,23 @@ __device__ __forceinline__ void tile_coords(const GemmGeom& g, int tile, int& mt
   }
 }
 
-// Epilogue interface (one object per epilogue thread, per tile):
-//   __device__ void begin(const Params&, int m_row, int nt);   // m_row: absolute row of D
+// Epilogue interface (one object per epilogue thread, per tile; every thread of the
+// warp calls each method, in step):
+//   __device__ void begin(const Params&, int m_row, int nt, const EpiCtx&);   // m_row: row of D
 //   __device__ void chunk(const Params&, int c, const uint32_t (&v)[32]);   // columns c*32..+31
 //   __device__ void end(const Params&);
 template <bool A_MN, bool B_MN, class Epi>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     k_tc_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-              GemmGeom g, typename Epi::Params ep, DevCtl ctl) {
+              const __grid_constant__ CUtensorMap tmC, GemmGeom g, typename Epi::Params ep,
+              DevCtl ctl) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sA = smem;                                  // kStages x 16 KiB
   uint8_t* sB = smem + kStages * kABytes;              // kStages x 32 KiB
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
+  uint8_t* sE = smem + kStages * kStageBytes;          // epilogue staging, 16 KiB
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sE + kEpiSmemBytes);
   // bars[0..S)   full      (TMA -> MMA)
   // bars[S..2S)  empty     (MMA -> TMA)
   // bars[2S..2S+2) acc_full  (MMA -> epilogue)
@@ -261,6 +276,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int lg = warp & 3;                 // TMEM lane group this warp may access
     const int row = lg * 32 + lane;
     const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(lg * 32) << 16);
+    const EpiCtx ectx{&tmC, smem_u32(sE + (warp - 2) * kEpiWarpBytes), lane};
     int local = 0;
     for (int tile = blockIdx.x; tile < n_tiles_total; tile += gridDim.x, ++local) {
       const int acc = local & 1;
@@ -274,7 +290,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int mt, nt;
       tile_coords(g, tile, mt, nt);
       Epi epi;
-      epi.begin(ep, mt * kBM + row, nt);
+      epi.begin(ep, mt * kBM + row, nt, ectx);
 #pragma unroll 1
       for (int c = 0; c < kBN / 32; ++c) {
         uint32_t v[32];
@@ -287,6 +303,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       epi.end(ep);
     }
   }
+
+  // Bulk stores an epilogue issued must finish before the CTA (and its shared
+  // memory) goes away; warps that issued none return at once.
+  if (warp >= 2 && lane == 0) bulk_wait_group<0>();
 
   // ---------------------------------------------------------------- teardown
   __syncthreads();
@@ -327,19 +347,21 @@ constexpr int kPStages = 6;
 constexpr int kPABytes = 128 * kBK * 2;            // 16 KiB: this CTA's 128 rows of A
 constexpr int kPBBytes = (kBN / 2) * kBK * 2;      // 16 KiB: this CTA's half of B
 constexpr int kPStageBytes = kPABytes + kPBBytes;
-constexpr int kPairSmemBytes = kPStages * kPStageBytes + 1024 + 256;
+constexpr int kPairSmemBytes = kPStages * kPStageBytes + kEpiSmemBytes + 1024 + 256;
 
 template <bool A_MN, bool B_MN, class Epi>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     k_tc_gemm_pair(const __grid_constant__ CUtensorMap tmA,
-                   const __grid_constant__ CUtensorMap tmB, GemmGeom g,
+                   const __grid_constant__ CUtensorMap tmB,
+                   const __grid_constant__ CUtensorMap tmC, GemmGeom g,
                    typename Epi::Params ep, DevCtl ctl) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + kPStages * kPABytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kPStages * kPStageBytes);
+  uint8_t* sE = smem + kPStages * kPStageBytes;        // epilogue staging, 16 KiB
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sE + kEpiSmemBytes);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kPStages + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -485,6 +507,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     const int row = static_cast<int>(rank) * 128 + lg * 32 + lane;
     const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(lg * 32) << 16);
     const uint32_t acce_leader = mapa_shared(acce0, 0);
+    const EpiCtx ectx{&tmC, smem_u32(sE + (warp - 2) * kEpiWarpBytes), lane};
     int local = 0;
     for (int tile = pair; tile < n_tiles_total; tile += n_pairs, ++local) {
       const int acc = local & 1;
@@ -498,7 +521,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       int mt, nt;
       tile_coords(g, tile, mt, nt);
       Epi epi;
-      epi.begin(ep, mt * kPairM + row, nt);
+      epi.begin(ep, mt * kPairM + row, nt, ectx);
 #pragma unroll 1
       for (int c = 0; c < kBN / 32; ++c) {
         uint32_t v[32];
@@ -511,6 +534,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       epi.end(ep);
     }
   }
+
+  // Bulk stores an epilogue issued must finish before the CTA (and its shared
+  // memory) goes away; warps that issued none return at once.
+  if (warp >= 2 && lane == 0) bulk_wait_group<0>();
 
   // ---------------------------------------------------------------- teardown
   __syncthreads();
