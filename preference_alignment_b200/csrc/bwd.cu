@@ -29,6 +29,7 @@ constexpr float kLog2eB = 1.4426950408889634f;
 // Two staging buffers per warp: a buffer is refilled only after the store issued
 // from it two chunks earlier has finished reading it.
 struct EpiGrad {
+  static constexpr bool kStaging = true;   // stores through TMA staging buffers
   struct Params {
     const int* y;
     const float* lse;
@@ -91,6 +92,7 @@ struct EpiGrad {
 
 // ------------------------------------------------------------------ dH rows epilogue
 struct EpiRows {
+  static constexpr bool kStaging = false;   // stores through TMA staging buffers
   struct Params {
     const int* dst;        // packed position -> flat row r * L + t
     float* out;            // dH [R * L, d]
@@ -134,6 +136,7 @@ struct EpiRows {
 
 // ------------------------------------------------------------------ dW epilogue
 struct EpiDW {
+  static constexpr bool kStaging = false;   // stores through TMA staging buffers
   struct Params {
     float* out;            // dW [V, d]
     int V, d, accumulate;

@@ -80,6 +80,7 @@ cudaError_t launch_prep(const uint16_t* H, const int* tokens, const Sched& s, in
 // ------------------------------------------------------------------ GEMM epilogue: online LSE
 // One thread = one packed position (accumulator row), 256 vocab columns per tile.
 struct EpiLSE {
+  static constexpr bool kStaging = false;   // stores through TMA staging buffers
   struct Params {
     const int* y;
     float2* part;

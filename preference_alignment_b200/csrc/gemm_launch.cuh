@@ -54,10 +54,10 @@ cudaError_t launch_gemm(const CUtensorMap& mapA, const CUtensorMap& mapB, const 
   const int k_blocks = (K + kBK - 1) / kBK;
   if (((gemm_variant() >> kind) & 1) == 0) {
     auto kern = k_tc_gemm_pair<A_MN, B_MN, Epi>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kPairSmemBytes);
+    constexpr int smem = pair_smem_bytes<Epi>();
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    const int clusters = max_pair_clusters(kern, kPairSmemBytes);
+    const int clusters = max_pair_clusters(kern, smem);
     if (clusters > 0) {
       GemmGeom g{(M + kPairM - 1) / kPairM, n_tiles, k_blocks, order, group > 0 ? group : 1,
                  0, nullptr};
@@ -75,7 +75,7 @@ cudaError_t launch_gemm(const CUtensorMap& mapA, const CUtensorMap& mapB, const 
           g.sync = sync;
         }
       }
-      kern<<<2 * pairs, kGemmThreads, kPairSmemBytes, st>>>(mapA, mapB, mapC, g, p, ctl);
+      kern<<<2 * pairs, kGemmThreads, smem, st>>>(mapA, mapB, mapC, g, p, ctl);
       return cudaGetLastError();
     }
   }

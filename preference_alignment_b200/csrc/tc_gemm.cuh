@@ -343,11 +343,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 // No TMA load uses cluster multicast: each CTA reads only its own operand rows.
 // =====================================================================================
 constexpr int kPairM = 256;                        // rows of D per CTA pair
-constexpr int kPStages = 6;
 constexpr int kPABytes = 128 * kBK * 2;            // 16 KiB: this CTA's 128 rows of A
 constexpr int kPBBytes = (kBN / 2) * kBK * 2;      // 16 KiB: this CTA's half of B
 constexpr int kPStageBytes = kPABytes + kPBBytes;
-constexpr int kPairSmemBytes = kPStages * kPStageBytes + kEpiSmemBytes + 1024 + 256;
+// Pipeline depth: an epilogue that stores through TMA (Epi::kStaging) takes 16 KiB of
+// shared memory for its staging buffers and leaves room for 6 stages; the others get
+// a 7th stage, which hides more DRAM latency in the GEMMs whose operands miss L2.
+template <class Epi>
+constexpr int pair_stages() { return Epi::kStaging ? 6 : 7; }
+template <class Epi>
+constexpr int pair_smem_bytes() {
+  return pair_stages<Epi>() * kPStageBytes + (Epi::kStaging ? kEpiSmemBytes : 0) + 1024 + 256;
+}
 
 template <bool A_MN, bool B_MN, class Epi>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
@@ -355,13 +362,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                    const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmC, GemmGeom g,
                    typename Epi::Params ep, DevCtl ctl) {
+  constexpr int kPStages = pair_stages<Epi>();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + kPStages * kPABytes;
-  uint8_t* sE = smem + kPStages * kPStageBytes;        // epilogue staging, 16 KiB
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sE + kEpiSmemBytes);
+  uint8_t* sE = smem + kPStages * kPStageBytes;        // epilogue staging (Epi::kStaging)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sE + (Epi::kStaging ? kEpiSmemBytes : 0));
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kPStages + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
