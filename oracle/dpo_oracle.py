@@ -22,6 +22,9 @@ What it computes, step by step, in the order of the pages:
   ("DPO Training on GPU, in depth", sections "What one DPO step computes" and
   "A worked example of the numbers", and dpo_step in "A training configuration
   that fits").
+* Logits-mean metrics: the mean of the chosen rows' logits and of the rejected
+  rows' logits over every position and vocabulary entry ("Run Distributed
+  Full-Model DPO with PyTorch FSDP", Step 4 and "What to Watch Out For").
 * Backward of the loss through the sequence sums to the LM-head input H and
   weight W: dL/dz[t, v] = dL/dS_r * (onehot(y_t)[v] - softmax(z_t)[v]),
   dH[t] = dZ[t] . W, dW = sum_t dZ[t]^T h_t (chain rule on the definitions
@@ -257,6 +260,39 @@ def position_grad_h(h, W, target, coef):
     p = np.exp(z - z.max())
     p /= p.sum()
     return coef * (W[int(target)] - p @ W)
+
+
+# --------------------------------------------------------------------------------------
+# Logits-mean metrics
+# --------------------------------------------------------------------------------------
+def logits_mean(H, W, layout="halves"):
+    """Mean of the logits over the chosen rows and over the rejected rows.
+
+    The torchtune DPO loop of "Run Distributed Full-Model DPO with PyTorch FSDP"
+    splits the model's logits for the concatenated batch into the chosen and the
+    rejected halves (Step 4, concatenated_forward: every position of every row,
+    prompt and padding included, over the whole vocabulary) and logs their means as
+    policy_chosen_logits_mean and policy_rejected_logits_mean ("What to Watch Out
+    For"). Here the logits z = h_t . W^T of every position t of every row on one
+    side are formed chunk by chunk and averaged over rows x positions x vocabulary;
+    the layout says which rows are chosen (pair_rows). H: [R, L, d], W: [V, d].
+    Returns (chosen_mean, rejected_mean).
+    """
+    H = np.asarray(H, dtype=np.float64)
+    W = np.asarray(W, dtype=np.float64)
+    R, L, _ = H.shape
+    V = W.shape[0]
+    B = R // 2
+    means = []
+    for side in (0, 1):
+        sums = []
+        for pair in pair_rows(B, layout):
+            r = pair[side]
+            for t0 in range(0, L, CHUNK):
+                Z = H[r, t0:t0 + CHUNK] @ W.T
+                sums.append(math.fsum(Z.ravel()))
+        means.append(math.fsum(sums) / (B * L * V))
+    return means[0], means[1]
 
 
 # --------------------------------------------------------------------------------------

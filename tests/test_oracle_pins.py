@@ -371,3 +371,78 @@ def test_variant_row_coef_by_finite_differences(normalize, nll):
             fd = 0.5 * (O.dpo_loss(p1, ref, 0.1, layout, **kw)["loss"]
                         - O.dpo_loss(p2, ref, 0.1, layout, **kw)["loss"]) / (2 * eps)
             assert out["row_coef"][r] == pytest.approx(fd, rel=1e-6, abs=1e-12)
+
+
+# ---------------------------------------------------------------- logits-mean metrics
+def test_logits_mean_equal_vocab_rows_closed_form():
+    """Every vocabulary row equal to w makes every logit of position t equal h_t . w,
+    so each side's mean is the mean of h_t . w over its rows and ALL positions."""
+    rng = np.random.default_rng(40)
+    R, L, d, V = 6, 9, 5, 11
+    H = rng.normal(size=(R, L, d))
+    w = rng.normal(size=d)
+    W = np.tile(w, (V, 1))
+    for layout, chosen in (("halves", [0, 1, 2]), ("adjacent", [0, 2, 4])):
+        rejected = [r for r in range(R) if r not in chosen]
+        want = []
+        for rows in (chosen, rejected):
+            vals = [sum(H[r, t, k] * w[k] for k in range(d)) for r in rows for t in range(L)]
+            want.append(math.fsum(vals) / len(vals))
+        got = O.logits_mean(H, W, layout)
+        assert got[0] == pytest.approx(want[0], rel=1e-12, abs=1e-14)
+        assert got[1] == pytest.approx(want[1], rel=1e-12, abs=1e-14)
+
+
+def test_logits_mean_counts_prompt_and_pad_positions():
+    """A single nonzero hidden state at the last (pad, never scored) position of one
+    chosen row: the chosen mean is (h . sum_v W[v]) / (B L V), the rejected mean 0."""
+    R, L, d, V = 4, 6, 3, 5
+    H = np.zeros((R, L, d))
+    H[1, L - 1] = [2.0, -1.0, 0.5]
+    W = np.arange(V * d, dtype=np.float64).reshape(V, d) / 8.0 - 1.0
+    colsum = [sum(W[v, k] for v in range(V)) for k in range(d)]
+    want = sum(H[1, L - 1, k] * colsum[k] for k in range(d)) / (2 * L * V)
+    c, r = O.logits_mean(H, W, "halves")       # row 1 is chosen under halves (B = 2)
+    assert c == pytest.approx(want, rel=1e-14) and c != 0.0
+    assert r == 0.0
+    c, r = O.logits_mean(H, W, "adjacent")     # ... and rejected under adjacent pairs
+    assert c == 0.0 and r == pytest.approx(want, rel=1e-14)
+
+
+@pytest.mark.parametrize("seed", range(3))
+def test_logits_mean_bruteforce_50_digits(seed):
+    """Every logit summed in 50-digit decimal arithmetic, divided by the count."""
+    import decimal
+    rng = np.random.default_rng(50 + seed)
+    R, L, d, V = 4, 3, 3, 4
+    H = rng.normal(size=(R, L, d))
+    W = rng.normal(size=(V, d))
+    ctx = decimal.Context(prec=50)
+    D = decimal.Decimal
+    for layout, sides in (("halves", ([0, 1], [2, 3])), ("adjacent", ([0, 2], [1, 3]))):
+        got = O.logits_mean(H, W, layout)
+        for rows, g in zip(sides, got):
+            tot = D(0)
+            for r in rows:
+                for t in range(L):
+                    for v in range(V):
+                        for k in range(d):
+                            tot = ctx.add(tot, ctx.multiply(D(float(H[r, t, k])), D(float(W[v, k]))))
+            want = float(ctx.divide(tot, D(len(rows) * L * V)))
+            assert g == pytest.approx(want, rel=1e-13, abs=1e-15)
+
+
+def test_logits_mean_is_bilinear():
+    """sum_{t,v} h_t . W[v] = (sum_t h_t) . (sum_v W[v]): the mean follows from the
+    two sums, and scaling H or W scales it."""
+    rng = np.random.default_rng(41)
+    R, L, d, V = 4, 300, 7, 13          # L > 256: more than one position chunk per row
+    H = rng.normal(size=(R, L, d))
+    W = rng.normal(size=(V, d))
+    c, r = O.logits_mean(H, W)
+    u_c, u_r = H[:2].reshape(-1, d).sum(0), H[2:].reshape(-1, d).sum(0)
+    s = W.sum(0)
+    assert c == pytest.approx(float(u_c @ s) / (2 * L * V), rel=1e-10)
+    assert r == pytest.approx(float(u_r @ s) / (2 * L * V), rel=1e-10)
+    c2, r2 = O.logits_mean(3.0 * H, -0.5 * W)
+    assert c2 == pytest.approx(-1.5 * c, rel=1e-12) and r2 == pytest.approx(-1.5 * r, rel=1e-12)
