@@ -471,6 +471,23 @@ def run_ours(args):
     h2d = H_host.numel() * 2 + tok_host.numel() * 4
     d2h = (w.R if fwd_only else 2 + 3 * B) * 4
 
+    # ------------------------------------------------------------ logits-mean metrics
+    # dpo_logits_mean (not part of the step): two HBM-bound column sums (W, then each
+    # side's H rows) and a dot product; algorithmic bytes = W + H read once.
+    lm_means = torch.empty(2, device=dev)
+    for _ in range(3):
+        libdpo.logits_mean(bp, w.layout, lm_means, ws, stream=sp)
+    lm_reps = 10
+    l0 = torch.cuda.Event(enable_timing=True)
+    l1 = torch.cuda.Event(enable_timing=True)
+    l0.record(stream)
+    for _ in range(lm_reps):
+        libdpo.logits_mean(bp, w.layout, lm_means, ws, stream=sp)
+    l1.record(stream)
+    torch.cuda.synchronize(dev)
+    lm_ms = l0.elapsed_time(l1) / lm_reps
+    lm_bytes = 2 * (w.V * w.d + w.R * w.L * w.d)
+
     # ------------------------------------------------------------ same-box cuBLAS reference
     cublas = None
     if not args.no_cublas_reference:
@@ -496,6 +513,7 @@ def run_ours(args):
     alg_flop = (1 if fwd_only else 4) * gemm_flop          # policy fwd, ref fwd, dH, dW
     exe_flop = (1 if fwd_only else 5) * gemm_flop          # + backward logit recompute
     sustained = float(peaks.get("bf16_tflops_sustained", PEAKS_FALLBACK["bf16_tflops_sustained"]))
+    hbm_peak = float(peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"]))
     # dominant kernel: the forward LSE GEMM (two launches per step), timed by the events
     # around the reference dpo_seq_logprobs call (the call also runs the small prep,
     # combine and row-sum kernels, so the figure is a slight underestimate)
@@ -537,6 +555,11 @@ def run_ours(args):
             "clocks": clk,
             "cpu_baseline": cpu,
             "cublas_same_box": cublas,
+            "logits_mean_metric": {"ms": lm_ms, "bytes": lm_bytes,
+                                   "GB/s": lm_bytes / (lm_ms / 1e3) / 1e9,
+                                   "frac": lm_bytes / (lm_ms / 1e3) / 1e9 / hbm_peak,
+                                   "peak_gbs": hbm_peak, "bound": "hbm",
+                                   "note": "dpo_logits_mean, not part of the step; W and H read once"},
             "peak_device_bytes": torch.cuda.max_memory_allocated(dev),
             "logits_fp32_bytes_avoided": 4 * Nc * w.V,
         }

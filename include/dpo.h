@@ -172,6 +172,26 @@ dpo_status dpo_backward(const dpo_batch* batch, const float* lse_state, const fl
                         float* dH, float* dW, int accumulate_dW, void* ws, size_t ws_bytes,
                         void* stream);
 
+/* Logits-mean metrics: the mean of the logits z = h_t . W^T over every position
+ * (prompt, completion and padding) of the chosen rows, and separately of the
+ * rejected rows, over the whole vocabulary -- the policy_chosen_logits_mean and
+ * policy_rejected_logits_mean the torchtune DPO loop logs ("Run Distributed
+ * Full-Model DPO with PyTorch FSDP", Step 4 splits the logits of every position
+ * into the two halves; "What to Watch Out For" names the metrics).
+ *   batch    as for dpo_seq_logprobs; every position of every row counts, so
+ *            prompt_len / completion_len are checked but do not change the result;
+ *            R must be even
+ *   layout   which rows are chosen: DPO_PAIRS_HALVES (rows [0, R/2)) or
+ *            DPO_PAIRS_ADJACENT (even rows)
+ *   means    device [2] fp32, out: {chosen mean, rejected mean}
+ *   ws       device workspace, >= fwd_bytes of dpo_workspace_size, 256-byte aligned
+ * The logits are not formed: sum_{t,v} z_tv = (sum_t h_t) . (sum_v W[v]), so the
+ * call reads W and H once (column sums in fp64, fixed order: the same result on
+ * every run). Errors: DPO_ERR_INVALID_ARG (odd R, bad layout, NULL means, or any
+ * batch check of dpo_seq_logprobs), DPO_ERR_WORKSPACE, DPO_ERR_CUDA. */
+dpo_status dpo_logits_mean(const dpo_batch* batch, int32_t layout, float* means, void* ws,
+                           size_t ws_bytes, void* stream);
+
 /* Size of the scratch array built into the library for dpo_seq_logprobs_noalloc. */
 #define DPO_NOALLOC_SCRATCH_BYTES (32u << 20)
 

@@ -163,7 +163,8 @@ dpo_status make_plan(const dpo_batch* b, Plan* p) {
   p->off_part = take(sizeof(float2) * static_cast<size_t>(p->S) * p->ldp);
   p->off_zy = take(sizeof(float) * p->ldp);
   p->off_lp = take(sizeof(float) * p->ldp);
-  p->fwd_total = o;
+  // the forward workspace also serves dpo_logits_mean
+  p->fwd_total = std::max(o, align_up(logits_mean_bytes(b->d), kAlign));
 
   o = p->prefix;
   p->ldG = bf16 ? static_cast<long long>(align_up(b->V, 8)) : b->V;
@@ -400,6 +401,22 @@ dpo_status dpo_backward(const dpo_batch* batch, const float* lse_state, const fl
     }
   }
   return DPO_OK;
+}
+
+dpo_status dpo_logits_mean(const dpo_batch* batch, int32_t layout, float* means, void* ws,
+                           size_t ws_bytes, void* stream) {
+  Plan p;
+  dpo_status s = make_plan(batch, &p);
+  if (s != DPO_OK) return s;
+  if (p.R % 2 != 0 || means == nullptr ||
+      (layout != DPO_PAIRS_HALVES && layout != DPO_PAIRS_ADJACENT))
+    return DPO_ERR_INVALID_ARG;
+  if (!ws_ok(ws, ws_bytes, align_up(logits_mean_bytes(p.d), kAlign))) return DPO_ERR_WORKSPACE;
+  DevInfo di;
+  if ((s = device_info(&di)) != DPO_OK) return s;
+  return cuda_status(launch_logits_mean(batch->H, batch->W, p.dtype == DPO_BF16, p.R, p.L, p.d,
+                                        p.V, layout == DPO_PAIRS_ADJACENT ? 1 : 0, ws, means,
+                                        di.sms, static_cast<cudaStream_t>(stream)));
 }
 
 dpo_status dpo_check(void* stream) {

@@ -113,4 +113,11 @@ int gemm_variant();
 // Bounded-wait self-test: one CTA waits on an mbarrier nothing arrives on.
 cudaError_t launch_wait_selftest(const DevCtl& ctl, cudaStream_t st);
 
+// Logits-mean metrics (fp64 column sums of W and of each side's H rows, then their
+// dot products): means[0] chosen, means[1] rejected. ws: logits_mean_bytes(d).
+int logits_mean_splits(int d);
+size_t logits_mean_bytes(int d);
+cudaError_t launch_logits_mean(const void* H, const void* W, bool bf16, int R, int L, int d, int V,
+                               int adjacent, void* ws, float* means, int sms, cudaStream_t st);
+
 }  // namespace dpo

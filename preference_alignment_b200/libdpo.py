@@ -206,6 +206,19 @@ def backward(batch: BatchArgs, lse_state, row_coef, dH, dW, accumulate_dW: bool,
                                _nbytes(ws, ws_bytes), _stream(stream)), "dpo_backward")
 
 
+def logits_mean(batch: BatchArgs, layout, means, ws, ws_bytes=None, stream=None):
+    """dpo_logits_mean: means (device float32 [2]) = mean logit of the chosen rows and of the
+    rejected rows over every position and vocabulary entry."""
+    lib = load()
+    fn = lib.dpo_logits_mean
+    fn.argtypes = [ctypes.POINTER(Batch), ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p,
+                   ctypes.c_size_t, ctypes.c_void_p]
+    fn.restype = ctypes.c_int
+    lay = LAYOUTS[layout] if isinstance(layout, str) else int(layout)
+    _check(fn(ctypes.byref(batch.c), lay, _ptr(means), _ptr(ws), _nbytes(ws, ws_bytes),
+              _stream(stream)), "dpo_logits_mean")
+
+
 def selftest_wait_timeout(budget_ms: int, stream=None):
     """Launch the bounded-wait self-test (records DPO_ERR_TIMEOUT after budget_ms)."""
     lib = load()

@@ -151,3 +151,24 @@ def test_loss_ex_rejects_bad_options(lib, kw):
     with pytest.raises(libdpo.DpoError) as e:
         libdpo.loss_ex(2, "halves", FAKE, FAKE, 0.1, 1.0, FAKE, **kw)
     assert e.value.status == libdpo.ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("kw,layout,means,ws,code", [
+    (dict(R=3, P=[4, 4, 4], C=[10, 10, 10]), "halves", FAKE, FAKE, libdpo.ERR_INVALID_ARG),  # odd R
+    (dict(), 5, FAKE, FAKE, libdpo.ERR_INVALID_ARG),                                     # layout
+    (dict(), "halves", None, FAKE, libdpo.ERR_INVALID_ARG),                              # no output
+    (dict(dtype="f16"), "halves", FAKE, FAKE, libdpo.ERR_UNSUPPORTED),
+    (dict(), "halves", FAKE, FAKE + 16, libdpo.ERR_WORKSPACE),                           # misaligned
+    (dict(), "halves", FAKE, None, libdpo.ERR_WORKSPACE),
+])
+def test_logits_mean_rejects(lib, kw, layout, means, ws, code):
+    with pytest.raises(libdpo.DpoError) as e:
+        libdpo.logits_mean(_batch(**kw), layout, means, ws, ws_bytes=1 << 30)
+    assert e.value.status == code
+
+
+def test_forward_workspace_covers_the_logits_mean(lib):
+    # d = 65536 with a single scored position: the column-sum partials set the size
+    f, _, _ = libdpo.workspace_size(_batch(R=2, L=4, d=65536, V=16, P=[1, 1], C=[1, 0]))
+    slabs, groups = 65536 // 256, 65536 // 32
+    assert f >= (3 * (1024 // slabs) * 65536 + 2 * groups) * 8
