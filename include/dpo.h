@@ -172,6 +172,59 @@ dpo_status dpo_backward(const dpo_batch* batch, const float* lse_state, const fl
                         float* dH, float* dW, int accumulate_dW, void* ws, size_t ws_bytes,
                         void* stream);
 
+/* ---- Vocabulary-parallel head ----------------------------------------------
+ * W split by vocabulary rows across ranks, every rank holding the same batch (the
+ * vocabulary-parallel alternative to data parallelism for a head too large to
+ * replicate; [V, d] rows stay where they are). Per step, on every rank:
+ *   1. dpo_shard_logprob_parts on its rows -> per-position (lse_k, z_y,k);
+ *   2. all-gather those [Nc] vectors across the ranks, in shard order;
+ *   3. dpo_shard_combine -> the full-vocabulary sums, log-probs and lse_state,
+ *      identical on every rank;
+ *   4. (policy) dpo_shard_backward with the global lse_state -> this rank's dW
+ *      rows and a partial dH; all-reduce (sum) the partial dH across the ranks.
+ * The library makes no collective call: the caller moves the buffers (NCCL).
+ * Shard k's W is rows [offset, offset + V) of the full [total, d] head; shards
+ * must not overlap and must cover [0, total). */
+typedef struct {
+  int32_t offset;   /* first vocabulary row of this shard in the full head */
+  int32_t total;    /* vocabulary size of the full head (<= 2^24) */
+} dpo_vocab_shard;
+
+/* Step 1: the forward of dpo_seq_logprobs over this shard's rows only.
+ *   batch      the shard: W = its [V, d] rows, V = its row count; tokens are ids in
+ *              the full vocabulary (a token outside [0, total) is a bad target)
+ *   shard_lse  device [Nc] fp32, out: log sum_{v in shard} exp(z_v) per scored position
+ *   shard_zy   device [Nc] fp32, out: z of the target if this shard holds it, else -inf
+ *   ws         device workspace, >= fwd_bytes of dpo_workspace_size(batch)
+ * Nc = sum of completion_len. Errors: those of dpo_seq_logprobs, and
+ * DPO_ERR_INVALID_ARG for a shard outside [0, total). */
+dpo_status dpo_shard_logprob_parts(const dpo_batch* batch, const dpo_vocab_shard* shard,
+                                   float* shard_lse, float* shard_zy, void* ws, size_t ws_bytes,
+                                   void* stream);
+
+/* Step 3: merge the gathered parts of n_shards shards (row k = shard k):
+ *   shard_lse, shard_zy  device [n_shards, Nc] fp32 (all-gather of step 1's outputs)
+ *   seq_logp, tok_logp, lse_state  as dpo_seq_logprobs (tok_logp, lse_state may be NULL)
+ *   ws   device workspace, >= fwd_bytes of dpo_workspace_size(batch)
+ * lse = M + log sum_k exp(lse_k - M) in fp64, shards in index order, so every rank
+ * that merges the same gathered values gets the same bits; a bad target scores 0.
+ * batch is any shard's batch (its rows and tokens are used; W is not read). */
+dpo_status dpo_shard_combine(const dpo_batch* batch, int32_t vocab_total, int32_t n_shards,
+                             const float* shard_lse, const float* shard_zy, float* seq_logp,
+                             float* tok_logp, float* lse_state, void* ws, size_t ws_bytes,
+                             void* stream);
+
+/* Step 4: dpo_backward over this shard's rows, with lse_state from step 3:
+ * dz = row_coef (onehot - softmax) on the shard's columns (the softmax uses the
+ * full-vocabulary lse), dH_part = dz . W_shard (device [R, L, d] fp32, fully
+ * written; the sum over shards is dH), dW_shard (device [V, d] fp32, written or
+ * accumulated) = this shard's rows of dW. ws: >= bwd_min_bytes of
+ * dpo_workspace_size(batch). dH_part may be NULL. */
+dpo_status dpo_shard_backward(const dpo_batch* batch, const dpo_vocab_shard* shard,
+                              const float* lse_state, const float* row_coef, float* dH_part,
+                              float* dW_shard, int accumulate_dW, void* ws, size_t ws_bytes,
+                              void* stream);
+
 /* Logits-mean metrics: the mean of the logits z = h_t . W^T over every position
  * (prompt, completion and padding) of the chosen rows, and separately of the
  * rejected rows, over the whole vocabulary -- the policy_chosen_logits_mean and

@@ -97,6 +97,7 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct Plan {
   int R = 0, L = 0, d = 0, V = 0, dtype = 0;
+  int v0 = 0, Vtot = 0;                // W holds vocabulary rows [v0, v0 + V) of Vtot
   int Nc = 0;
   std::vector<int> row_start;          // [R + 1]
   // common prefix of both workspaces
@@ -128,6 +129,8 @@ dpo_status make_plan(const dpo_batch* b, Plan* p) {
   p->L = b->L;
   p->d = b->d;
   p->V = b->V;
+  p->v0 = 0;
+  p->Vtot = b->V;
   p->dtype = b->dtype;
   p->row_start.assign(b->R + 1, 0);
   long long nc = 0;
@@ -177,6 +180,16 @@ dpo_status make_plan(const dpo_batch* b, Plan* p) {
   return DPO_OK;
 }
 
+// The batch's W is vocabulary rows [offset, offset + V) of a head of `total` rows.
+dpo_status apply_shard(const dpo_vocab_shard* sh, Plan* p) {
+  if (sh == nullptr || sh->offset < 0 || sh->total < 1 || sh->total > (1 << 24) ||
+      static_cast<long long>(sh->offset) + p->V > sh->total)
+    return DPO_ERR_INVALID_ARG;
+  p->v0 = sh->offset;
+  p->Vtot = sh->total;
+  return DPO_OK;
+}
+
 Sched sched_of(const Plan& p, void* ws) {
   uint8_t* w = static_cast<uint8_t*>(ws);
   Sched s;
@@ -193,7 +206,7 @@ dpo_status cuda_status(cudaError_t e) { return e == cudaSuccess ? DPO_OK : DPO_E
 
 // Upload the row table and build the scored-position tables (+ packed H for bf16).
 dpo_status stage_schedule(const Plan& p, const dpo_batch* b, void* ws, const DevCtl& ctl,
-                          cudaStream_t st) {
+                          cudaStream_t st, bool pack = true) {
   uint8_t* w = static_cast<uint8_t*>(ws);
   std::vector<RowChunk> chunks((p.R + kRowChunk - 1) / kRowChunk);
   for (size_t c = 0; c < chunks.size(); ++c) {
@@ -210,117 +223,50 @@ dpo_status stage_schedule(const Plan& p, const dpo_batch* b, void* ws, const Dev
                                        reinterpret_cast<int*>(w + p.off_P), st);
     if (e != cudaSuccess) return DPO_ERR_CUDA;
   }
-  uint16_t* Hp = p.dtype == DPO_BF16 ? reinterpret_cast<uint16_t*>(w + p.off_hp) : nullptr;
+  uint16_t* Hp = pack && p.dtype == DPO_BF16 ? reinterpret_cast<uint16_t*>(w + p.off_hp) : nullptr;
   return cuda_status(launch_prep(static_cast<const uint16_t*>(b->H), b->tokens, sched_of(p, ws),
-                                 p.R, p.L, p.d, p.V, p.Nc, Hp, ctl, st));
+                                 p.R, p.L, p.d, p.V, p.v0, p.Vtot, p.Nc, Hp, ctl, st));
 }
 
 bool ws_ok(const void* ws, size_t have, size_t need) {
   return ws != nullptr && have >= need && reinterpret_cast<uintptr_t>(ws) % kAlign == 0;
 }
 
-}  // namespace
-
-int dpo::gemm_variant() { return g_gemm_variant.load(); }
-
-extern "C" {
-
-dpo_status dpo_workspace_size(const dpo_batch* batch, size_t* fwd_bytes, size_t* bwd_bytes,
-                              size_t* bwd_min_bytes) {
-  Plan p;
-  const dpo_status s = make_plan(batch, &p);
-  if (s != DPO_OK) return s;
-  if (fwd_bytes) *fwd_bytes = p.fwd_total;
-  if (bwd_bytes) *bwd_bytes = p.bwd_total;
-  if (bwd_min_bytes) *bwd_min_bytes = p.bwd_min;
-  return DPO_OK;
-}
-
-dpo_status dpo_seq_logprobs(const dpo_batch* batch, int want_grad, float* seq_logp,
-                            float* tok_logp, float* lse_state, void* ws, size_t ws_bytes,
-                            void* stream) {
-  Plan p;
-  dpo_status s = make_plan(batch, &p);
-  if (s != DPO_OK) return s;
-  if (seq_logp == nullptr || (want_grad && lse_state == nullptr)) return DPO_ERR_INVALID_ARG;
-  if (!ws_ok(ws, ws_bytes, p.fwd_total)) return DPO_ERR_WORKSPACE;
-  DevInfo di;
-  if ((s = device_info(&di)) != DPO_OK) return s;
-  const DevCtl ctl = make_ctl(di);
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
+// Schedule, LM-head GEMM with the online log-sum-exp, and the combine over the
+// vocabulary tiles: lp in the workspace; lse and the target logit (-inf when the
+// target is not in this call's rows) when asked.
+dpo_status forward_core(const Plan& p, const dpo_batch* batch, void* ws, float* lse_out,
+                        float* zy_out, const DevInfo& di, const DevCtl& ctl, cudaStream_t st) {
   uint8_t* w = static_cast<uint8_t*>(ws);
-
-  if ((s = stage_schedule(p, batch, ws, ctl, st)) != DPO_OK) return s;
+  dpo_status s = stage_schedule(p, batch, ws, ctl, st);
+  if (s != DPO_OK) return s;
   const Sched sc = sched_of(p, ws);
   float2* part = reinterpret_cast<float2*>(w + p.off_part);
   float* zy = reinterpret_cast<float*>(w + p.off_zy);
   float* lp = reinterpret_cast<float*>(w + p.off_lp);
-
-  if (p.Nc > 0) {
-    if (p.dtype == DPO_BF16) {
-      CUtensorMap mA, mB;
-      if (!make_map(&mA, w + p.off_hp, p.d, p.Nc, 2ull * p.d, kBK, kBoxRows) ||
-          !make_map(&mB, batch->W, p.d, p.V, 2ull * p.d, kBK, kBoxRows))
-        return DPO_ERR_CUDA;
-      if (launch_fwd_lse(mA, mB, p.Nc, p.V, p.d, sc.y, part, p.ldp, zy, di.sms, sc.sync, ctl,
-                         st) != cudaSuccess)
-        return DPO_ERR_CUDA;
-    } else {
-      if (launch_f32_fwd(static_cast<const float*>(batch->H), static_cast<const float*>(batch->W),
-                         sc, p.Nc, p.d, p.V, part, zy, st) != cudaSuccess)
-        return DPO_ERR_CUDA;
-    }
-    if (launch_combine(part, p.ldp, p.S, zy, sc.y, p.Nc, lp, want_grad ? lse_state : nullptr,
-                       st) != cudaSuccess)
+  if (p.Nc == 0) return DPO_OK;
+  if (p.dtype == DPO_BF16) {
+    CUtensorMap mA, mB;
+    if (!make_map(&mA, w + p.off_hp, p.d, p.Nc, 2ull * p.d, kBK, kBoxRows) ||
+        !make_map(&mB, batch->W, p.d, p.V, 2ull * p.d, kBK, kBoxRows))
+      return DPO_ERR_CUDA;
+    if (launch_fwd_lse(mA, mB, p.Nc, p.V, p.d, sc.y, part, p.ldp, zy, di.sms, sc.sync, ctl, st) !=
+        cudaSuccess)
+      return DPO_ERR_CUDA;
+  } else {
+    if (launch_f32_fwd(static_cast<const float*>(batch->H), static_cast<const float*>(batch->W),
+                       sc, p.Nc, p.d, p.V, part, zy, st) != cudaSuccess)
       return DPO_ERR_CUDA;
   }
-  return cuda_status(launch_rowsum(lp, sc.row_start, sc.prompt, p.R, p.L, seq_logp, tok_logp, st));
+  return cuda_status(launch_combine(part, p.ldp, p.S, zy, sc.y, p.Nc, lp, lse_out, zy_out, st));
 }
 
-dpo_status dpo_loss(int32_t B, int32_t layout, const float* pol, const float* ref, float beta,
-                    float grad_scale, float* loss, float* accuracy, float* margins,
-                    float* chosen_rewards, float* rejected_rewards, float* weights,
-                    float* row_coef, void* stream) {
-  if (B < 1 || B > (1 << 28) || (layout != DPO_PAIRS_HALVES && layout != DPO_PAIRS_ADJACENT))
-    return DPO_ERR_INVALID_ARG;
-  if (pol == nullptr || ref == nullptr || loss == nullptr) return DPO_ERR_INVALID_ARG;
-  if (!(beta > 0.f) || !std::isfinite(beta) || !std::isfinite(grad_scale))
-    return DPO_ERR_INVALID_ARG;
-  return cuda_status(launch_loss(B, layout, pol, ref, beta, grad_scale, 0, 0.0, nullptr, loss,
-                                 accuracy, margins, chosen_rewards, rejected_rewards, weights,
-                                 row_coef, nullptr, static_cast<cudaStream_t>(stream)));
-}
-
-dpo_status dpo_loss_ex(int32_t B, int32_t layout, const float* pol, const float* ref, float beta,
-                       float grad_scale, const dpo_loss_options* opt, float* loss, float* accuracy,
-                       float* margins, float* chosen_rewards, float* rejected_rewards,
-                       float* weights, float* row_coef, float* nll, void* stream) {
-  if (B < 1 || B > (1 << 28) || (layout != DPO_PAIRS_HALVES && layout != DPO_PAIRS_ADJACENT))
-    return DPO_ERR_INVALID_ARG;
-  if (pol == nullptr || ref == nullptr || loss == nullptr) return DPO_ERR_INVALID_ARG;
-  if (!(beta > 0.f) || !std::isfinite(beta) || !std::isfinite(grad_scale))
-    return DPO_ERR_INVALID_ARG;
-  int normalize = 0;
-  float nll_weight = 0.f;
-  const int32_t* clen = nullptr;
-  if (opt != nullptr) {
-    normalize = opt->normalize ? 1 : 0;
-    nll_weight = opt->nll_weight;
-    clen = opt->completion_len;
-    if (!std::isfinite(nll_weight) || nll_weight < 0.f) return DPO_ERR_INVALID_ARG;
-    if ((normalize || nll_weight > 0.f) && clen == nullptr) return DPO_ERR_INVALID_ARG;
-  }
-  return cuda_status(launch_loss(B, layout, pol, ref, beta, grad_scale, normalize, nll_weight,
-                                 clen, loss, accuracy, margins, chosen_rewards, rejected_rewards,
-                                 weights, row_coef, nll, static_cast<cudaStream_t>(stream)));
-}
-
-dpo_status dpo_backward(const dpo_batch* batch, const float* lse_state, const float* row_coef,
-                        float* dH, float* dW, int accumulate_dW, void* ws, size_t ws_bytes,
-                        void* stream) {
-  Plan p;
-  dpo_status s = make_plan(batch, &p);
-  if (s != DPO_OK) return s;
+// Backward of sum_r row_coef[r] S_r for this call's vocabulary rows: dz chunks,
+// dH (fully written) and dW (written or accumulated).
+dpo_status backward_core(const Plan& p, const dpo_batch* batch, const float* lse_state,
+                         const float* row_coef, float* dH, float* dW, int accumulate_dW, void* ws,
+                         size_t ws_bytes, void* stream) {
+  dpo_status s = DPO_OK;
   if ((p.Nc > 0 && lse_state == nullptr) || row_coef == nullptr || dW == nullptr)
     return DPO_ERR_INVALID_ARG;
   if (!ws_ok(ws, ws_bytes, p.bwd_min)) return DPO_ERR_WORKSPACE;
@@ -401,6 +347,148 @@ dpo_status dpo_backward(const dpo_batch* batch, const float* lse_state, const fl
     }
   }
   return DPO_OK;
+}
+
+}  // namespace
+
+int dpo::gemm_variant() { return g_gemm_variant.load(); }
+
+extern "C" {
+
+dpo_status dpo_workspace_size(const dpo_batch* batch, size_t* fwd_bytes, size_t* bwd_bytes,
+                              size_t* bwd_min_bytes) {
+  Plan p;
+  const dpo_status s = make_plan(batch, &p);
+  if (s != DPO_OK) return s;
+  if (fwd_bytes) *fwd_bytes = p.fwd_total;
+  if (bwd_bytes) *bwd_bytes = p.bwd_total;
+  if (bwd_min_bytes) *bwd_min_bytes = p.bwd_min;
+  return DPO_OK;
+}
+
+dpo_status dpo_seq_logprobs(const dpo_batch* batch, int want_grad, float* seq_logp,
+                            float* tok_logp, float* lse_state, void* ws, size_t ws_bytes,
+                            void* stream) {
+  Plan p;
+  dpo_status s = make_plan(batch, &p);
+  if (s != DPO_OK) return s;
+  if (seq_logp == nullptr || (want_grad && lse_state == nullptr)) return DPO_ERR_INVALID_ARG;
+  if (!ws_ok(ws, ws_bytes, p.fwd_total)) return DPO_ERR_WORKSPACE;
+  DevInfo di;
+  if ((s = device_info(&di)) != DPO_OK) return s;
+  const DevCtl ctl = make_ctl(di);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+
+  if ((s = forward_core(p, batch, ws, want_grad ? lse_state : nullptr, nullptr, di, ctl, st)) !=
+      DPO_OK)
+    return s;
+  const Sched sc = sched_of(p, ws);
+  float* lp = reinterpret_cast<float*>(w + p.off_lp);
+  return cuda_status(launch_rowsum(lp, sc.row_start, sc.prompt, p.R, p.L, seq_logp, tok_logp, st));
+}
+
+dpo_status dpo_shard_logprob_parts(const dpo_batch* batch, const dpo_vocab_shard* shard,
+                                   float* shard_lse, float* shard_zy, void* ws, size_t ws_bytes,
+                                   void* stream) {
+  Plan p;
+  dpo_status s = make_plan(batch, &p);
+  if (s != DPO_OK) return s;
+  if ((s = apply_shard(shard, &p)) != DPO_OK) return s;
+  if (shard_lse == nullptr || shard_zy == nullptr) return DPO_ERR_INVALID_ARG;
+  if (!ws_ok(ws, ws_bytes, p.fwd_total)) return DPO_ERR_WORKSPACE;
+  DevInfo di;
+  if ((s = device_info(&di)) != DPO_OK) return s;
+  return forward_core(p, batch, ws, shard_lse, shard_zy, di, make_ctl(di),
+                      static_cast<cudaStream_t>(stream));
+}
+
+dpo_status dpo_shard_combine(const dpo_batch* batch, int32_t vocab_total, int32_t n_shards,
+                             const float* shard_lse, const float* shard_zy, float* seq_logp,
+                             float* tok_logp, float* lse_state, void* ws, size_t ws_bytes,
+                             void* stream) {
+  Plan p;
+  dpo_status s = make_plan(batch, &p);
+  if (s != DPO_OK) return s;
+  if (vocab_total < p.V || vocab_total > (1 << 24) || n_shards < 1 || n_shards > vocab_total ||
+      seq_logp == nullptr || (p.Nc > 0 && (shard_lse == nullptr || shard_zy == nullptr)))
+    return DPO_ERR_INVALID_ARG;
+  if (!ws_ok(ws, ws_bytes, p.fwd_total)) return DPO_ERR_WORKSPACE;
+  DevInfo di;
+  if ((s = device_info(&di)) != DPO_OK) return s;
+  const DevCtl ctl = make_ctl(di);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // targets classified against the whole head: valid or bad, never "elsewhere"
+  Plan q = p;
+  q.v0 = 0;
+  q.V = vocab_total;
+  q.Vtot = vocab_total;
+  if ((s = stage_schedule(q, batch, ws, ctl, st, false)) != DPO_OK) return s;
+  const Sched sc = sched_of(p, ws);
+  float* lp = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + p.off_lp);
+  if (launch_shard_combine(shard_lse, shard_zy, n_shards, p.Nc, sc.y, lp, lse_state, st) !=
+      cudaSuccess)
+    return DPO_ERR_CUDA;
+  return cuda_status(launch_rowsum(lp, sc.row_start, sc.prompt, p.R, p.L, seq_logp, tok_logp, st));
+}
+
+dpo_status dpo_loss(int32_t B, int32_t layout, const float* pol, const float* ref, float beta,
+                    float grad_scale, float* loss, float* accuracy, float* margins,
+                    float* chosen_rewards, float* rejected_rewards, float* weights,
+                    float* row_coef, void* stream) {
+  if (B < 1 || B > (1 << 28) || (layout != DPO_PAIRS_HALVES && layout != DPO_PAIRS_ADJACENT))
+    return DPO_ERR_INVALID_ARG;
+  if (pol == nullptr || ref == nullptr || loss == nullptr) return DPO_ERR_INVALID_ARG;
+  if (!(beta > 0.f) || !std::isfinite(beta) || !std::isfinite(grad_scale))
+    return DPO_ERR_INVALID_ARG;
+  return cuda_status(launch_loss(B, layout, pol, ref, beta, grad_scale, 0, 0.0, nullptr, loss,
+                                 accuracy, margins, chosen_rewards, rejected_rewards, weights,
+                                 row_coef, nullptr, static_cast<cudaStream_t>(stream)));
+}
+
+dpo_status dpo_loss_ex(int32_t B, int32_t layout, const float* pol, const float* ref, float beta,
+                       float grad_scale, const dpo_loss_options* opt, float* loss, float* accuracy,
+                       float* margins, float* chosen_rewards, float* rejected_rewards,
+                       float* weights, float* row_coef, float* nll, void* stream) {
+  if (B < 1 || B > (1 << 28) || (layout != DPO_PAIRS_HALVES && layout != DPO_PAIRS_ADJACENT))
+    return DPO_ERR_INVALID_ARG;
+  if (pol == nullptr || ref == nullptr || loss == nullptr) return DPO_ERR_INVALID_ARG;
+  if (!(beta > 0.f) || !std::isfinite(beta) || !std::isfinite(grad_scale))
+    return DPO_ERR_INVALID_ARG;
+  int normalize = 0;
+  float nll_weight = 0.f;
+  const int32_t* clen = nullptr;
+  if (opt != nullptr) {
+    normalize = opt->normalize ? 1 : 0;
+    nll_weight = opt->nll_weight;
+    clen = opt->completion_len;
+    if (!std::isfinite(nll_weight) || nll_weight < 0.f) return DPO_ERR_INVALID_ARG;
+    if ((normalize || nll_weight > 0.f) && clen == nullptr) return DPO_ERR_INVALID_ARG;
+  }
+  return cuda_status(launch_loss(B, layout, pol, ref, beta, grad_scale, normalize, nll_weight,
+                                 clen, loss, accuracy, margins, chosen_rewards, rejected_rewards,
+                                 weights, row_coef, nll, static_cast<cudaStream_t>(stream)));
+}
+
+dpo_status dpo_backward(const dpo_batch* batch, const float* lse_state, const float* row_coef,
+                        float* dH, float* dW, int accumulate_dW, void* ws, size_t ws_bytes,
+                        void* stream) {
+  Plan p;
+  const dpo_status s = make_plan(batch, &p);
+  if (s != DPO_OK) return s;
+  return backward_core(p, batch, lse_state, row_coef, dH, dW, accumulate_dW, ws, ws_bytes, stream);
+}
+
+dpo_status dpo_shard_backward(const dpo_batch* batch, const dpo_vocab_shard* shard,
+                              const float* lse_state, const float* row_coef, float* dH_part,
+                              float* dW_shard, int accumulate_dW, void* ws, size_t ws_bytes,
+                              void* stream) {
+  Plan p;
+  dpo_status s = make_plan(batch, &p);
+  if (s != DPO_OK) return s;
+  if ((s = apply_shard(shard, &p)) != DPO_OK) return s;
+  return backward_core(p, batch, lse_state, row_coef, dH_part, dW_shard, accumulate_dW, ws,
+                       ws_bytes, stream);
 }
 
 dpo_status dpo_logits_mean(const dpo_batch* batch, int32_t layout, float* means, void* ws,

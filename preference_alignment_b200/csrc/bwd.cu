@@ -54,7 +54,9 @@ struct EpiGrad {
       const int y = __ldg(p.y + gt);
       yl = y - vbase;
       nl2 = -__ldg(p.lse + gt) * kLog2eB;
-      cf = y >= 0 ? __ldg(p.coef + __ldg(p.rowid + gt)) : 0.f;  // bad target: no gradient
+      // bad target: no gradient; a target in another vocabulary shard keeps the
+      // softmax term (yl never matches a column of this call)
+      cf = y != kTargetBad ? __ldg(p.coef + __ldg(p.rowid + gt)) : 0.f;
     }
   }
 
@@ -92,7 +94,7 @@ struct EpiGrad {
 
 // ------------------------------------------------------------------ dH rows epilogue
 struct EpiRows {
-  static constexpr bool kStaging = false;   // stores through TMA staging buffers
+  static constexpr bool kStaging = false;   // stores go straight to global memory
   struct Params {
     const int* dst;        // packed position -> flat row r * L + t
     float* out;            // dH [R * L, d]
@@ -136,7 +138,7 @@ struct EpiRows {
 
 // ------------------------------------------------------------------ dW epilogue
 struct EpiDW {
-  static constexpr bool kStaging = false;   // stores through TMA staging buffers
+  static constexpr bool kStaging = false;   // stores go straight to global memory
   struct Params {
     float* out;            // dW [V, d]
     int V, d, accumulate;

@@ -90,7 +90,7 @@ __global__ void __launch_bounds__(256) k_f32_grad(const float* __restrict__ H,
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const float* h = H + static_cast<long long>(s.dst[gt]) * d;
   const int y = s.y[gt];
-  const float cf = y >= 0 ? coef[s.rowid[gt]] : 0.f;
+  const float cf = y != kTargetBad ? coef[s.rowid[gt]] : 0.f;
   const float l = lse[gt];
   float* g = G + static_cast<long long>(i) * V;
   for (int v = warp; v < V; v += 8) {

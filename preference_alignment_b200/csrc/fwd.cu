@@ -42,7 +42,7 @@ cudaError_t launch_upload_rows(const RowChunk& rc, int* row_start, int* prompt,
 // its position t = P_r - 1 + (i - row_start[r]) and target tokens[r, t + 1].
 __global__ void __launch_bounds__(256) k_prep(const uint16_t* __restrict__ H,
                                               const int* __restrict__ tokens, Sched s, int R,
-                                              int L, int d, int V, int Nc,
+                                              int L, int d, int V, int v0, int Vtot, int Nc,
                                               uint16_t* __restrict__ Hp, DevCtl ctl) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int i = blockIdx.x * 8 + warp;
@@ -57,9 +57,10 @@ __global__ void __launch_bounds__(256) k_prep(const uint16_t* __restrict__ H,
   const long long src = static_cast<long long>(r) * L + t;
   if (lane == 0) {
     const int tgt = __ldg(tokens + src + 1);
-    const bool ok = tgt >= 0 && tgt < V;
+    const bool ok = tgt >= 0 && tgt < Vtot;
     if (!ok) record_status(ctl, kStatusBadTarget);
-    s.y[i] = ok ? tgt : -1;
+    const int yl = tgt - v0;            // column in this call's vocabulary rows [v0, v0 + V)
+    s.y[i] = !ok ? kTargetBad : (yl >= 0 && yl < V ? yl : kTargetElsewhere);
     s.dst[i] = static_cast<int>(src);
     s.rowid[i] = r;
   }
@@ -71,16 +72,17 @@ __global__ void __launch_bounds__(256) k_prep(const uint16_t* __restrict__ H,
 }
 
 cudaError_t launch_prep(const uint16_t* H, const int* tokens, const Sched& s, int R, int L, int d,
-                        int V, int Nc, uint16_t* Hp, const DevCtl& ctl, cudaStream_t st) {
+                        int V, int v0, int Vtot, int Nc, uint16_t* Hp, const DevCtl& ctl,
+                        cudaStream_t st) {
   if (Nc == 0) return cudaSuccess;
-  k_prep<<<(Nc + 7) / 8, 256, 0, st>>>(H, tokens, s, R, L, d, V, Nc, Hp, ctl);
+  k_prep<<<(Nc + 7) / 8, 256, 0, st>>>(H, tokens, s, R, L, d, V, v0, Vtot, Nc, Hp, ctl);
   return cudaGetLastError();
 }
 
 // ------------------------------------------------------------------ GEMM epilogue: online LSE
 // One thread = one packed position (accumulator row), 256 vocab columns per tile.
 struct EpiLSE {
-  static constexpr bool kStaging = false;   // stores through TMA staging buffers
+  static constexpr bool kStaging = false;   // stores go straight to global memory
   struct Params {
     const int* y;
     float2* part;
@@ -96,7 +98,7 @@ struct EpiLSE {
     tok = m_row;
     valid = tok < p.Nc;
     const int vbase = nt * kBN;
-    yl = valid ? __ldg(p.y + tok) - vbase : -1;   // y = -1 (bad target) never matches
+    yl = valid ? __ldg(p.y + tok) - vbase : -1;   // negative targets never match
     vlim = p.V - vbase;
     mx = -INFINITY;
     s = 0.f;
@@ -170,7 +172,8 @@ __global__ void __launch_bounds__(256) k_combine(const float2* __restrict__ part
                                                  const float* __restrict__ zy,
                                                  const int* __restrict__ y, int Nc,
                                                  float* __restrict__ lp,
-                                                 float* __restrict__ lse_out) {
+                                                 float* __restrict__ lse_out,
+                                                 float* __restrict__ zy_out) {
   __shared__ float sm[8][32], ss[8][32];
   const int g = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int i = blockIdx.x * 32 + lane;
@@ -199,15 +202,57 @@ __global__ void __launch_bounds__(256) k_combine(const float2* __restrict__ part
     float Mt = sm[0][lane], St = ss[0][lane];
     for (int h = 1; h < 8; ++h) lse_merge(Mt, St, sm[h][lane], ss[h][lane]);
     const float lse = Mt + logf(St);
-    lp[i] = (__ldg(y + i) >= 0) ? __ldg(zy + i) - lse : 0.f;
+    const bool here = __ldg(y + i) >= 0;
+    lp[i] = here ? __ldg(zy + i) - lse : 0.f;
     if (lse_out != nullptr) lse_out[i] = lse;
+    if (zy_out != nullptr) zy_out[i] = here ? __ldg(zy + i) : -INFINITY;
   }
 }
 
 cudaError_t launch_combine(const float2* part, int ldp, int S, const float* zy, const int* y,
-                           int Nc, float* lp, float* lse_out, cudaStream_t st) {
+                           int Nc, float* lp, float* lse_out, float* zy_out, cudaStream_t st) {
   if (Nc == 0) return cudaSuccess;
-  k_combine<<<(Nc + 31) / 32, 256, 0, st>>>(part, ldp, S, zy, y, Nc, lp, lse_out);
+  k_combine<<<(Nc + 31) / 32, 256, 0, st>>>(part, ldp, S, zy, y, Nc, lp, lse_out, zy_out);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ vocabulary shards
+// Merge the per-shard results of each position (shards in index order, fp64):
+//   lse = M + log(sum_k exp(lse_k - M)),  M = max_k lse_k
+//   z_y = the one finite shard value (the shard that holds the target)
+//   lp  = z_y - lse, or 0 for a bad target (y = kTargetBad)
+// One thread per position; the shard order is fixed, so every rank that merges the
+// same gathered values gets the same bits.
+__global__ void __launch_bounds__(256) k_shard_combine(const float* __restrict__ lse_parts,
+                                                       const float* __restrict__ zy_parts,
+                                                       int n_shards, int Nc,
+                                                       const int* __restrict__ y,
+                                                       float* __restrict__ lp,
+                                                       float* __restrict__ lse_out) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= Nc) return;
+  double M = -INFINITY;
+  float zyv = -INFINITY;
+  for (int k = 0; k < n_shards; ++k) {
+    M = fmax(M, static_cast<double>(__ldg(lse_parts + static_cast<long long>(k) * Nc + i)));
+    zyv = fmaxf(zyv, __ldg(zy_parts + static_cast<long long>(k) * Nc + i));
+  }
+  double S = 0.0;
+  for (int k = 0; k < n_shards; ++k) {
+    const double l = __ldg(lse_parts + static_cast<long long>(k) * Nc + i);
+    if (l != -INFINITY) S += exp(l - M);
+  }
+  const float lse = static_cast<float>(M + log(S));
+  lp[i] = __ldg(y + i) == kTargetBad ? 0.f : zyv - lse;
+  if (lse_out != nullptr) lse_out[i] = lse;
+}
+
+cudaError_t launch_shard_combine(const float* lse_parts, const float* zy_parts, int n_shards,
+                                 int Nc, const int* y, float* lp, float* lse_out,
+                                 cudaStream_t st) {
+  if (Nc == 0) return cudaSuccess;
+  k_shard_combine<<<(Nc + 255) / 256, 256, 0, st>>>(lse_parts, zy_parts, n_shards, Nc, y, lp,
+                                                    lse_out);
   return cudaGetLastError();
 }
 

@@ -32,6 +32,11 @@ struct RowChunk {
   int P[kRowChunk];               // prompt length of each row
 };
 
+// Target of a scored position, as k_prep stores it: the column in the call's
+// vocabulary rows, or one of these (neither matches a vocabulary column).
+constexpr int kTargetBad = -1;         // token outside [0, total vocabulary): scored 0, no gradient
+constexpr int kTargetElsewhere = -2;   // valid token held by another vocabulary shard
+
 // Device views of the per-call schedule held in the workspace.
 struct Sched {
   const int* row_start;   // [R + 1] packed offset of row r's first scored position
@@ -46,9 +51,11 @@ cudaError_t launch_upload_rows(const RowChunk& rc, int* row_start, int* prompt,
                                cudaStream_t st);
 
 // Scored-position tables (y, dst, rowid) and, when Hp != nullptr, the packed
-// bf16 copy of the scored H rows.
+// bf16 copy of the scored H rows. The call's W holds vocabulary rows [v0, v0 + V) of
+// a head of Vtot rows (v0 = 0, Vtot = V for the whole head).
 cudaError_t launch_prep(const uint16_t* H, const int* tokens, const Sched& s, int R, int L, int d,
-                        int V, int Nc, uint16_t* Hp, const DevCtl& ctl, cudaStream_t st);
+                        int V, int v0, int Vtot, int Nc, uint16_t* Hp, const DevCtl& ctl,
+                        cudaStream_t st);
 
 // Forward GEMM with the online log-sum-exp epilogue (bf16, tcgen05).
 //   part[nt * ldp + i] = (max, sum exp(z - max)) of vocab tile nt for packed position i
@@ -57,9 +64,15 @@ cudaError_t launch_fwd_lse(const CUtensorMap& mapA, const CUtensorMap& mapB, int
                            int d, const int* y, float2* part, int ldp, float* zy, int grid,
                            int* sync, const DevCtl& ctl, cudaStream_t st);
 
-// Combine the vocab-tile partials of each position into lse and lp = zy - lse.
+// Combine the vocab-tile partials of each position into lse and lp = zy - lse;
+// optionally the target logit, -inf when the target is not in the call's rows.
 cudaError_t launch_combine(const float2* part, int ldp, int S, const float* zy, const int* y,
-                           int Nc, float* lp, float* lse_out, cudaStream_t st);
+                           int Nc, float* lp, float* lse_out, float* zy_out, cudaStream_t st);
+
+// Merge [n_shards, Nc] per-shard (lse, z_y) into lp and lse (shards in index order).
+cudaError_t launch_shard_combine(const float* lse_parts, const float* zy_parts, int n_shards,
+                                 int Nc, const int* y, float* lp, float* lse_out,
+                                 cudaStream_t st);
 
 // Per-row fp64 sum of lp over the row's scored positions; optional [R, L] token output.
 cudaError_t launch_rowsum(const float* lp, const int* row_start, const int* prompt, int R, int L,

@@ -206,6 +206,52 @@ def backward(batch: BatchArgs, lse_state, row_coef, dH, dW, accumulate_dW: bool,
                                _nbytes(ws, ws_bytes), _stream(stream)), "dpo_backward")
 
 
+class VocabShard(ctypes.Structure):
+    _fields_ = [("offset", ctypes.c_int32), ("total", ctypes.c_int32)]
+
+
+def shard_logprob_parts(batch: BatchArgs, offset: int, total: int, shard_lse, shard_zy, ws,
+                        ws_bytes=None, stream=None):
+    """dpo_shard_logprob_parts: per-position (lse, target logit or -inf) over one shard's rows."""
+    lib = load()
+    fn = lib.dpo_shard_logprob_parts
+    vp = ctypes.c_void_p
+    fn.argtypes = [ctypes.POINTER(Batch), ctypes.POINTER(VocabShard), vp, vp, vp, ctypes.c_size_t, vp]
+    fn.restype = ctypes.c_int
+    sh = VocabShard(int(offset), int(total))
+    _check(fn(ctypes.byref(batch.c), ctypes.byref(sh), _ptr(shard_lse), _ptr(shard_zy), _ptr(ws),
+              _nbytes(ws, ws_bytes), _stream(stream)), "dpo_shard_logprob_parts")
+
+
+def shard_combine(batch: BatchArgs, total: int, n_shards: int, shard_lse, shard_zy, seq_logp,
+                  tok_logp, lse_state, ws, ws_bytes=None, stream=None):
+    """dpo_shard_combine: merge gathered [n_shards, Nc] parts into sums, log-probs and lse."""
+    lib = load()
+    fn = lib.dpo_shard_combine
+    vp = ctypes.c_void_p
+    fn.argtypes = [ctypes.POINTER(Batch), ctypes.c_int32, ctypes.c_int32, vp, vp, vp, vp, vp, vp,
+                   ctypes.c_size_t, vp]
+    fn.restype = ctypes.c_int
+    _check(fn(ctypes.byref(batch.c), int(total), int(n_shards), _ptr(shard_lse), _ptr(shard_zy),
+              _ptr(seq_logp), _ptr(tok_logp), _ptr(lse_state), _ptr(ws), _nbytes(ws, ws_bytes),
+              _stream(stream)), "dpo_shard_combine")
+
+
+def shard_backward(batch: BatchArgs, offset: int, total: int, lse_state, row_coef, dH_part,
+                   dW_shard, accumulate_dW: bool, ws, ws_bytes=None, stream=None):
+    """dpo_shard_backward: this shard's dW rows and a partial dH (summed over shards = dH)."""
+    lib = load()
+    fn = lib.dpo_shard_backward
+    vp = ctypes.c_void_p
+    fn.argtypes = [ctypes.POINTER(Batch), ctypes.POINTER(VocabShard), vp, vp, vp, vp, ctypes.c_int,
+                   vp, ctypes.c_size_t, vp]
+    fn.restype = ctypes.c_int
+    sh = VocabShard(int(offset), int(total))
+    _check(fn(ctypes.byref(batch.c), ctypes.byref(sh), _ptr(lse_state), _ptr(row_coef),
+              _ptr(dH_part), _ptr(dW_shard), 1 if accumulate_dW else 0, _ptr(ws),
+              _nbytes(ws, ws_bytes), _stream(stream)), "dpo_shard_backward")
+
+
 def logits_mean(batch: BatchArgs, layout, means, ws, ws_bytes=None, stream=None):
     """dpo_logits_mean: means (device float32 [2]) = mean logit of the chosen rows and of the
     rejected rows over every position and vocabulary entry."""

@@ -172,3 +172,35 @@ def test_forward_workspace_covers_the_logits_mean(lib):
     f, _, _ = libdpo.workspace_size(_batch(R=2, L=4, d=65536, V=16, P=[1, 1], C=[1, 0]))
     slabs, groups = 65536 // 256, 65536 // 32
     assert f >= (3 * (1024 // slabs) * 65536 + 2 * groups) * 8
+
+
+@pytest.mark.parametrize("offset,total,code", [
+    (-1, 100, libdpo.ERR_INVALID_ARG),
+    (1, 100, libdpo.ERR_INVALID_ARG),            # offset + V = 101 > total
+    (0, (1 << 24) + 1, libdpo.ERR_INVALID_ARG),
+    (0, 0, libdpo.ERR_INVALID_ARG),
+])
+def test_shard_calls_reject_windows_outside_the_head(lib, offset, total, code):
+    b = _batch(V=100)
+    with pytest.raises(libdpo.DpoError) as e:
+        libdpo.shard_logprob_parts(b, offset, total, FAKE, FAKE, FAKE, ws_bytes=1 << 30)
+    assert e.value.status == code
+    with pytest.raises(libdpo.DpoError) as e:
+        libdpo.shard_backward(b, offset, total, FAKE, FAKE, None, FAKE, False, FAKE,
+                              ws_bytes=1 << 30)
+    assert e.value.status == code
+
+
+def test_shard_calls_reject_missing_outputs_and_workspace(lib):
+    b = _batch(V=100)
+    for lse, zy in ((None, FAKE), (FAKE, None)):
+        with pytest.raises(libdpo.DpoError) as e:
+            libdpo.shard_logprob_parts(b, 0, 300, lse, zy, FAKE, ws_bytes=1 << 30)
+        assert e.value.status == libdpo.ERR_INVALID_ARG
+    with pytest.raises(libdpo.DpoError) as e:
+        libdpo.shard_logprob_parts(b, 0, 300, FAKE, FAKE, FAKE + 16, ws_bytes=1 << 30)
+    assert e.value.status == libdpo.ERR_WORKSPACE
+    for total, n, seq in ((99, 1, FAKE), (300, 0, FAKE), (300, 2, None), ((1 << 24) + 1, 2, FAKE)):
+        with pytest.raises(libdpo.DpoError) as e:
+            libdpo.shard_combine(b, total, n, FAKE, FAKE, seq, None, None, FAKE, ws_bytes=1 << 30)
+        assert e.value.status == libdpo.ERR_INVALID_ARG
