@@ -7,7 +7,8 @@
 //   sum_{t, v} z_tv = sum_k (sum_t h_tk) (sum_v W_vk),
 // so each side needs the column sums of its H rows and of W, and one dot product.
 // The work is two HBM-bound column reductions (W read once, H once) and a tiny
-// finishing kernel; every sum runs in fp64 in a fixed order, so the result is the
+// finishing kernel. Each lane adds groups of 8 (bf16) or 4 (fp32) rows in fp32 and
+// the group sums in fp64; every reduction has a fixed order, so the result is the
 // same for every run.
 #include "internal.h"
 
@@ -32,7 +33,8 @@ struct RowMap {
 };
 
 // One row's 8 columns, loaded raw (loads of several rows are issued before any is
-// converted, to keep enough bytes in flight) and added in fp64.
+// converted, to keep enough bytes in flight); a group of rows is added in fp32, the
+// group sums and the tail rows in fp64.
 template <typename T>
 struct Raw8;
 
@@ -42,6 +44,14 @@ struct Raw8<uint16_t> {
   uint4 v;
   __device__ __forceinline__ void load(const uint16_t* p) {
     v = __ldg(reinterpret_cast<const uint4*>(p));
+  }
+  __device__ __forceinline__ void add_f32(float (&f)[8]) const {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      f[2 * j] += __uint_as_float(w[j] << 16);
+      f[2 * j + 1] += __uint_as_float(w[j] & 0xffff0000u);
+    }
   }
   __device__ __forceinline__ void add_to(double (&acc)[8]) const {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -60,6 +70,10 @@ struct Raw8<float> {
   __device__ __forceinline__ void load(const float* p) {
     a = __ldg(reinterpret_cast<const float4*>(p));
     b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  }
+  __device__ __forceinline__ void add_f32(float (&f)[8]) const {
+    f[0] += a.x; f[1] += a.y; f[2] += a.z; f[3] += a.w;
+    f[4] += b.x; f[5] += b.y; f[6] += b.z; f[7] += b.w;
   }
   __device__ __forceinline__ void add_to(double (&acc)[8]) const {
     acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
@@ -114,8 +128,15 @@ __global__ void __launch_bounds__(kWarps * 32, 3)
       Raw8<T> x[U];
 #pragma unroll
       for (int u = 0; u < U; ++u) x[u].load(X + map(i + u * kWarps) * d + col);
+      // the U rows are added in fp32 first (one fp64 conversion per U values: the
+      // conversion, not HBM, limits the kernel at power-capped clocks otherwise)
+      float f[8];
 #pragma unroll
-      for (int u = 0; u < U; ++u) x[u].add_to(acc);
+      for (int j = 0; j < 8; ++j) f[j] = 0.f;
+#pragma unroll
+      for (int u = 0; u < U; ++u) x[u].add_f32(f);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc[j] += static_cast<double>(f[j]);
     }
     for (; i < r1; i += kWarps) {
       Raw8<T> x;
