@@ -122,3 +122,31 @@ def test_logits_mean_llama8b_head_bilinear_form():
         want.append(float(u @ s) / (R // 2 * L * w.V))
         scale.append(_bound_terms(u, s, A, S) / (R // 2 * L * w.V))
     _assert_close(got, want, scale)
+
+
+def test_logits_mean_largest_hidden_size():
+    """d = 65,536: 256 column slabs, one row split each."""
+    w = WL.make_custom(R=2, L=8, d=65536, V=64, dtype="bf16", seed=8, prompt_range=(1, 1),
+                       min_completion=1)
+    H, W = WL.widen(w.H, "bf16"), WL.widen(w.W, "bf16")
+    got, _, _, _ = _run(w, "halves")
+    _assert_close(got, O.logits_mean(H, W, "halves"), _scale(H, W, "halves"))
+
+
+def test_logits_mean_largest_vocabulary():
+    """V = 2^24 rows of W in one column slab: the bilinear form, block by block."""
+    w = WL.make_custom(R=2, L=8, d=8, V=1 << 24, dtype="bf16", seed=9, prompt_range=(1, 1),
+                       min_completion=1)
+    got, _, _, _ = _run(w, "adjacent")
+    s, S = np.zeros(w.d), np.zeros(w.d)
+    for v0 in range(0, w.V, 1 << 20):
+        blk = WL.widen(w.W[v0:v0 + (1 << 20)], "bf16")
+        s += blk.sum(axis=0)
+        S += np.abs(blk).sum(axis=0)
+    H = WL.widen(w.H, "bf16")
+    want, scale = [], []
+    for rows in _side_rows(w.R, "adjacent"):
+        h = H[rows].reshape(-1, w.d)
+        want.append(float(h.sum(axis=0) @ s) / (w.L * w.V))
+        scale.append(_bound_terms(h.sum(axis=0), s, np.abs(h).sum(axis=0), S) / (w.L * w.V))
+    _assert_close(got, want, scale)
