@@ -346,11 +346,13 @@ constexpr int kPairM = 256;                        // rows of D per CTA pair
 constexpr int kPABytes = 128 * kBK * 2;            // 16 KiB: this CTA's 128 rows of A
 constexpr int kPBBytes = (kBN / 2) * kBK * 2;      // 16 KiB: this CTA's half of B
 constexpr int kPStageBytes = kPABytes + kPBBytes;
-// Pipeline depth: an epilogue that stores through TMA (Epi::kStaging) takes 16 KiB of
-// shared memory for its staging buffers and leaves room for 6 stages; the others get
-// a 7th stage, which hides more DRAM latency in the GEMMs whose operands miss L2.
+// Pipeline depth: 6 stages of 32 KiB for every epilogue (an epilogue that stores
+// through TMA, Epi::kStaging, adds 16 KiB of staging buffers). A 7th stage fits the
+// epilogues without staging and made the serialised GEMMs ~1 % faster under ncu, but
+// inside the power-capped step (same box, alternating runs at the Llama-3.1-8B head)
+// 6 stages were 0.2-2.3 % faster.
 template <class Epi>
-constexpr int pair_stages() { return Epi::kStaging ? 6 : 7; }
+constexpr int pair_stages() { return 6; }
 template <class Epi>
 constexpr int pair_smem_bytes() {
   return pair_stages<Epi>() * kPStageBytes + (Epi::kStaging ? kEpiSmemBytes : 0) + 1024 + 256;
