@@ -9,6 +9,7 @@
 #include <vector>
 
 #include <cudaTypedefs.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include "dpo.h"
 #include "internal.h"
@@ -20,6 +21,15 @@ __device__ int g_dpo_status_word = 0;
 namespace {
 
 using namespace dpo;
+
+// NVTX range around an entry point (names the call on profiler timelines; with no
+// tool attached the push/pop cost a few nanoseconds).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 constexpr size_t kAlign = 256;
 constexpr int kMinChunk = 128;   // smallest backward token chunk
@@ -369,6 +379,7 @@ dpo_status dpo_workspace_size(const dpo_batch* batch, size_t* fwd_bytes, size_t*
 dpo_status dpo_seq_logprobs(const dpo_batch* batch, int want_grad, float* seq_logp,
                             float* tok_logp, float* lse_state, void* ws, size_t ws_bytes,
                             void* stream) {
+  NvtxRange nvtx_range("dpo_seq_logprobs");
   Plan p;
   dpo_status s = make_plan(batch, &p);
   if (s != DPO_OK) return s;
@@ -391,6 +402,7 @@ dpo_status dpo_seq_logprobs(const dpo_batch* batch, int want_grad, float* seq_lo
 dpo_status dpo_shard_logprob_parts(const dpo_batch* batch, const dpo_vocab_shard* shard,
                                    float* shard_lse, float* shard_zy, void* ws, size_t ws_bytes,
                                    void* stream) {
+  NvtxRange nvtx_range("dpo_shard_logprob_parts");
   Plan p;
   dpo_status s = make_plan(batch, &p);
   if (s != DPO_OK) return s;
@@ -407,6 +419,7 @@ dpo_status dpo_shard_combine(const dpo_batch* batch, int32_t vocab_total, int32_
                              const float* shard_lse, const float* shard_zy, float* seq_logp,
                              float* tok_logp, float* lse_state, void* ws, size_t ws_bytes,
                              void* stream) {
+  NvtxRange nvtx_range("dpo_shard_combine");
   Plan p;
   dpo_status s = make_plan(batch, &p);
   if (s != DPO_OK) return s;
@@ -436,6 +449,7 @@ dpo_status dpo_loss(int32_t B, int32_t layout, const float* pol, const float* re
                     float grad_scale, float* loss, float* accuracy, float* margins,
                     float* chosen_rewards, float* rejected_rewards, float* weights,
                     float* row_coef, void* stream) {
+  NvtxRange nvtx_range("dpo_loss");
   if (B < 1 || B > (1 << 28) || (layout != DPO_PAIRS_HALVES && layout != DPO_PAIRS_ADJACENT))
     return DPO_ERR_INVALID_ARG;
   if (pol == nullptr || ref == nullptr || loss == nullptr) return DPO_ERR_INVALID_ARG;
@@ -450,6 +464,7 @@ dpo_status dpo_loss_ex(int32_t B, int32_t layout, const float* pol, const float*
                        float grad_scale, const dpo_loss_options* opt, float* loss, float* accuracy,
                        float* margins, float* chosen_rewards, float* rejected_rewards,
                        float* weights, float* row_coef, float* nll, void* stream) {
+  NvtxRange nvtx_range("dpo_loss_ex");
   if (B < 1 || B > (1 << 28) || (layout != DPO_PAIRS_HALVES && layout != DPO_PAIRS_ADJACENT))
     return DPO_ERR_INVALID_ARG;
   if (pol == nullptr || ref == nullptr || loss == nullptr) return DPO_ERR_INVALID_ARG;
@@ -473,6 +488,7 @@ dpo_status dpo_loss_ex(int32_t B, int32_t layout, const float* pol, const float*
 dpo_status dpo_backward(const dpo_batch* batch, const float* lse_state, const float* row_coef,
                         float* dH, float* dW, int accumulate_dW, void* ws, size_t ws_bytes,
                         void* stream) {
+  NvtxRange nvtx_range("dpo_backward");
   Plan p;
   const dpo_status s = make_plan(batch, &p);
   if (s != DPO_OK) return s;
@@ -483,6 +499,7 @@ dpo_status dpo_shard_backward(const dpo_batch* batch, const dpo_vocab_shard* sha
                               const float* lse_state, const float* row_coef, float* dH_part,
                               float* dW_shard, int accumulate_dW, void* ws, size_t ws_bytes,
                               void* stream) {
+  NvtxRange nvtx_range("dpo_shard_backward");
   Plan p;
   dpo_status s = make_plan(batch, &p);
   if (s != DPO_OK) return s;
@@ -493,6 +510,7 @@ dpo_status dpo_shard_backward(const dpo_batch* batch, const dpo_vocab_shard* sha
 
 dpo_status dpo_logits_mean(const dpo_batch* batch, int32_t layout, float* means, void* ws,
                            size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_range("dpo_logits_mean");
   Plan p;
   dpo_status s = make_plan(batch, &p);
   if (s != DPO_OK) return s;
@@ -508,6 +526,7 @@ dpo_status dpo_logits_mean(const dpo_batch* batch, int32_t layout, float* means,
 }
 
 dpo_status dpo_check(void* stream) {
+  NvtxRange nvtx_range("dpo_check");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   DevInfo di;
   dpo_status s = device_info(&di);
@@ -522,6 +541,7 @@ dpo_status dpo_check(void* stream) {
 }
 
 dpo_status dpo_fingerprint(const void* data, size_t bytes, uint64_t* out, void* stream) {
+  NvtxRange nvtx_range("dpo_fingerprint");
   if (out == nullptr || reinterpret_cast<uintptr_t>(out) % 8 != 0) return DPO_ERR_INVALID_ARG;
   if (bytes > 0 && (data == nullptr || reinterpret_cast<uintptr_t>(data) % 16 != 0))
     return DPO_ERR_INVALID_ARG;
