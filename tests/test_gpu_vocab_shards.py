@@ -189,3 +189,52 @@ def test_llama8b_head_in_eight_shards():
     assert libdpo.check() == libdpo.OK
     assert rel_frob(np64(dH), np64(dH1)) <= 1e-3
     assert rel_frob(np64(dW), np64(dW1)) <= 1e-3
+
+
+def test_shard_calls_and_logits_mean_replay_from_a_cuda_graph():
+    """Two shards' parts, the merge, both shard backwards and the logits mean, captured
+    into one CUDA graph and replayed: the same outputs as the direct calls."""
+    import torch
+    w = WL.make_custom(R=4, L=160, d=256, V=1300, dtype="bf16", seed=76, prompt_range=(1, 60))
+    dw = DeviceWorkload(w)
+    shards = [(0, 768), (768, 532)]
+    nc = w.n_scored
+    bs = [_shard_batch(dw, o, n) for o, n in shards]
+    need = max(max(libdpo.workspace_size(b)[:2]) for b in bs)
+    wss = [dw.workspace(need) for _ in shards]
+    parts = torch.empty(2, len(shards), nc, device="cuda")
+    seq = torch.empty(w.R, device="cuda")
+    lse = torch.empty(nc, device="cuda")
+    coef = torch.linspace(-0.1, 0.1, w.R, device="cuda")
+    dHs = [torch.empty(w.R, w.L, w.d, device="cuda") for _ in shards]
+    dWs = [torch.empty(n, w.d, device="cuda") for _, n in shards]
+    means = torch.empty(2, device="cuda")
+    full = libdpo.BatchArgs(dw.H, dw.W, dw.tokens, w.prompt_len, w.completion_len, dtype="bf16")
+    ws_full = dw.workspace(libdpo.workspace_size(full)[0])
+
+    def run(stream):
+        for k, ((o, n), b) in enumerate(zip(shards, bs)):
+            libdpo.shard_logprob_parts(b, o, w.V, parts[0, k], parts[1, k], wss[k], stream=stream)
+        libdpo.shard_combine(bs[0], w.V, len(shards), parts[0], parts[1], seq, None, lse, wss[0],
+                             stream=stream)
+        for k, ((o, n), b) in enumerate(zip(shards, bs)):
+            libdpo.shard_backward(b, o, w.V, lse, coef, dHs[k], dWs[k], False, wss[k],
+                                  stream=stream)
+        libdpo.logits_mean(full, "halves", means, ws_full, stream=stream)
+
+    outs = [parts, seq, lse, *dHs, *dWs, means]
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        run(s.cuda_stream)
+    s.synchronize()
+    direct = [t.clone() for t in outs]
+    for t in outs:
+        t.fill_(float("nan"))
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        run(s.cuda_stream)
+    g.replay()
+    torch.cuda.synchronize()
+    assert libdpo.check() == libdpo.OK
+    for a, b in zip(direct, outs):
+        assert torch.equal(a, b)
