@@ -35,6 +35,7 @@ WORKLOAD = "llama8b"
 CONFIG_TEXT = ("Llama-3.1-8B head shape: 4 pairs -> 8 rows, seq 2048, prompt U{256..1024}, "
                "completion to >=95% fill, d=4096, V=128256, bf16; policy fwd+bwd, reference fwd")
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+DH_VOCAB_CHUNK = 16384   # vocabulary columns per dH GEMM launch in the library's backward
 
 
 # ------------------------------------------------------------------ helpers
@@ -372,11 +373,13 @@ def run_ours(args):
             DP.allreduce_step(dW, outs["loss"])
 
     # launches of our kernels per step: upload + prep + GEMM + combine + rowsum per forward,
-    # one loss kernel, upload + prep + 3 GEMMs for the backward (one token chunk: the
-    # workspace holds all Nc rows of dz)
+    # one loss kernel; the backward (one token chunk: the workspace holds all Nc rows of
+    # dz) runs upload + prep + the dz GEMM + one dH GEMM per DH_VOCAB_CHUNK vocabulary
+    # columns + the dW GEMM
     uploads = math.ceil(w.R / 1024)
     fwd_launches = uploads + 4
-    launches_per_step = (fwd_launches if fwd_only else 2 * fwd_launches + 1 + uploads + 4)
+    bwd_launches = uploads + 3 + math.ceil(w.V / DH_VOCAB_CHUNK)
+    launches_per_step = (fwd_launches if fwd_only else 2 * fwd_launches + 1 + bwd_launches)
 
     for _ in range(args.warmup):
         step()
