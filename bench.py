@@ -36,6 +36,7 @@ CONFIG_TEXT = ("Llama-3.1-8B head shape: 4 pairs -> 8 rows, seq 2048, prompt U{2
                "completion to >=95% fill, d=4096, V=128256, bf16; policy fwd+bwd, reference fwd")
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 DH_VOCAB_CHUNK = 16384   # vocabulary columns per dH GEMM launch in the library's backward
+                         # (vocabularies of at least 4 chunks; shorter ones: one launch)
 
 
 # ------------------------------------------------------------------ helpers
@@ -378,7 +379,8 @@ def run_ours(args):
     # columns + the dW GEMM
     uploads = math.ceil(w.R / 1024)
     fwd_launches = uploads + 4
-    bwd_launches = uploads + 3 + math.ceil(w.V / DH_VOCAB_CHUNK)
+    dh_launches = math.ceil(w.V / DH_VOCAB_CHUNK) if w.V >= 4 * DH_VOCAB_CHUNK else 1
+    bwd_launches = uploads + 3 + dh_launches
     launches_per_step = (fwd_launches if fwd_only else 2 * fwd_launches + 1 + bwd_launches)
 
     for _ in range(args.warmup):

@@ -325,10 +325,12 @@ dpo_status backward_core(const Plan& p, const dpo_batch* batch, const float* lse
       if (launch_bwd_grad(mHk, mWk, mGst, mc, p.V, p.d, tok0, sc.y, lse_state, row_coef,
                           sc.rowid, di.sms, sc.sync, ctl, st) != cudaSuccess)
         return DPO_ERR_CUDA;
-      // dH = dz . W reduces over the vocabulary: chunks of kDhVocabChunk columns, the
-      // later ones added to the rows by the epilogue.
-      for (int v0 = 0; dH != nullptr && v0 < p.V; v0 += kDhVocabChunk) {
-        const int vc = std::min(kDhVocabChunk, p.V - v0);
+      // dH = dz . W reduces over the vocabulary: one launch, or chunks of kDhVocabChunk
+      // columns for a long vocabulary (never longer than kMaxAccumK), the later ones
+      // added to the rows by the epilogue.
+      const int dh_chunk = p.V >= kDhChunkFrom ? kDhVocabChunk : kMaxAccumK;
+      for (int v0 = 0; dH != nullptr && v0 < p.V; v0 += dh_chunk) {
+        const int vc = std::min(dh_chunk, p.V - v0);
         CUtensorMap mGkc = mGk, mWmnc = mWmn;
         if (v0 > 0 || vc < p.V) {
           if (!make_map(&mGkc, G + v0, vc, mc, 2ull * p.ldG, kBK, kBoxRows) ||
