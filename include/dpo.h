@@ -302,9 +302,10 @@ dpo_status dpo_selftest_wait_timeout(uint32_t budget_ms, void* stream);
  * one bit per GEMM: bit 0 the forward (logits + log-sum-exp), bit 1 the backward's
  * logit recompute (dz), bit 2 dH = dz.W, bit 3 dW = dz^T.H. A clear bit runs that
  * GEMM on a pair of CTAs (tcgen05.mma.cta_group::2, 256 x 256 tiles) when the
- * device can co-schedule CTA pairs, else on one CTA; a set bit always runs it on
- * one CTA (128 x 256 tiles). Both give the same results within rounding. Default
- * 0. Returns the previous mask, or -1 for a value outside 0..15. */
+ * device can co-schedule CTA pairs, unless one CTA per 128 x 256 tile fills the
+ * GPU's waves more than 5 % better for that launch's shape; a set bit always runs
+ * it on one CTA. Both give the same results within rounding. Default 0. Returns
+ * the previous mask, or -1 for a value outside 0..15. */
 int32_t dpo_set_gemm_variant(int32_t variant);
 
 /* Static description of a status code. */

@@ -37,11 +37,29 @@ int max_pair_clusters(Kern kern, int smem_bytes) {
   return n;
 }
 
+// Fraction of a launch's row slots that hold real rows: M rows in tiles of tile_m,
+// times n_tiles, spread over `slots` concurrent tiles in whole waves (the ragged
+// last row tile and the partly idle last wave are the waste).
+inline double tile_fill(int M, int tile_m, int n_tiles, int slots) {
+  const long long tiles = static_cast<long long>((M + tile_m - 1) / tile_m) * n_tiles;
+  const long long waves = (tiles + slots - 1) / slots;
+  return static_cast<double>(M) * n_tiles / (static_cast<double>(waves) * slots * tile_m);
+}
+
+// A CTA pair does a 256-row tile ~3 % faster than two single CTAs do its halves
+// (measured under the power cap); the single-CTA kernel is chosen only when its
+// finer tiles fill the GPU's waves better by more than this margin.
+constexpr double kPairMargin = 1.05;
+
 // D[M x N] = A[M x K] . B[N x K]^T with the epilogue Epi; `order` picks the tile
 // raster (0: M fastest, 1: N fastest); `sms` is the device's SM count.
 // Raster: `order` as in GemmGeom (0, 1, or 2/3 grouped along M/N with `group`
 // 256-wide tiles per group; a group of 0 falls back to order 0).
-// `kind` (a GemmKind) selects this GEMM's bit of the dpo_set_gemm_variant mask.
+// `kind` (a GemmKind) selects this GEMM's bit of the dpo_set_gemm_variant mask: a set
+// bit forces the single-CTA kernel; a clear bit runs CTA pairs unless 128-row tiles
+// fill the waves clearly better (tile_fill), e.g. 4,648 rows x 8 column tiles: 152
+// pair tiles are 2.05 waves of 74 pairs (3 launched, 68 % full), 296 single tiles
+// exactly 2 waves of 148 CTAs.
 // mapC is the epilogue's store tensor map (epilogues that do not store through TMA
 // ignore it; pass any valid map).
 template <bool A_MN, bool B_MN, class Epi>
@@ -65,18 +83,22 @@ cudaError_t launch_gemm(const CUtensorMap& mapA, const CUtensorMap& mapB, const 
       int pairs = clusters < sms / 2 ? clusters : sms / 2;
       if (pairs > tiles) pairs = tiles;
       if (pairs < 1) pairs = 1;
-      if (epoch > 0 && sync != nullptr) {
-        // epochs this launch can reach; pacing stays off if the counters do not fit
-        const long long per_pair = static_cast<long long>((tiles + pairs - 1) / pairs) * k_blocks;
-        if (per_pair / epoch + 1 < sync_len) {
-          e = cudaMemsetAsync(sync, 0, sizeof(int) * (per_pair / epoch + 2), st);
-          if (e != cudaSuccess) return e;
-          g.epoch = epoch;
-          g.sync = sync;
+      const bool single_fills_better =
+          tile_fill(M, kBM, n_tiles, sms) > kPairMargin * tile_fill(M, kPairM, n_tiles, pairs);
+      if (!single_fills_better) {
+        if (epoch > 0 && sync != nullptr) {
+          // epochs this launch can reach; pacing stays off if the counters do not fit
+          const long long per_pair = static_cast<long long>((tiles + pairs - 1) / pairs) * k_blocks;
+          if (per_pair / epoch + 1 < sync_len) {
+            e = cudaMemsetAsync(sync, 0, sizeof(int) * (per_pair / epoch + 2), st);
+            if (e != cudaSuccess) return e;
+            g.epoch = epoch;
+            g.sync = sync;
+          }
         }
+        kern<<<2 * pairs, kGemmThreads, smem, st>>>(mapA, mapB, mapC, g, p, ctl);
+        return cudaGetLastError();
       }
-      kern<<<2 * pairs, kGemmThreads, smem, st>>>(mapA, mapB, mapC, g, p, ctl);
-      return cudaGetLastError();
     }
   }
   auto kern = k_tc_gemm<A_MN, B_MN, Epi>;
