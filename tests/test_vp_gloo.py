@@ -146,3 +146,22 @@ def test_two_rank_vocab_parallel_equals_unsharded_oracle():
     dW = np.concatenate([res[r][4] for r in range(WORLD)])
     assert res[1][0] == res[0][4].shape[0]               # shards are contiguous, in rank order
     np.testing.assert_allclose(dW, oW, rtol=1e-9, atol=1e-12)
+
+
+def test_shard_range_partitions_the_vocabulary():
+    """Shards are disjoint, in rank order, cover [0, total), are non-empty, and are whole
+    256-row tiles (but the last) whenever that leaves every rank a row."""
+    from preference_alignment_b200 import vp
+    for total in (1, 7, 255, 256, 1000, 32000, 128256, 151936, 1 << 24):
+        for world in (1, 2, 3, 4, 7, 8, 64):
+            if world > total:
+                continue
+            parts = [vp.shard_range(total, world, r) for r in range(world)]
+            at = 0
+            for off, n in parts:
+                assert off == at and n >= 1
+                at += n
+            assert at == total
+            per = -(-(-(-total // world)) // 256) * 256
+            if per * (world - 1) < total:
+                assert all(n % 256 == 0 for _, n in parts[:-1])
