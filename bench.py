@@ -167,11 +167,18 @@ PROFILED_SOURCES = ["preference_alignment_b200/csrc/" + f for f in
 
 
 def kernel_source_hash():
+    """Hash of the profiled kernel sources' code: comments, blank lines and trailing
+    spaces are dropped first, so only a change of code makes the counters stale."""
     import hashlib
+    import re
     h = hashlib.sha256()
     for f in PROFILED_SOURCES:
-        with open(os.path.join(ROOT, f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, f)) as fh:
+            text = fh.read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        code = "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
+        h.update(code.encode())
     return h.hexdigest()[:16]
 
 

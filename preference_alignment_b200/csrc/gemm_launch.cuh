@@ -1,6 +1,7 @@
 // Host-side launch of the tcgen05 GEMM kernels (included by the .cu files that
 // instantiate them). The CTA-pair kernel is the default; the single-CTA kernel
-// is used when the device cannot co-schedule CTA pairs.
+// is used when the device cannot co-schedule CTA pairs, when its 128-row tiles
+// fill the waves clearly better, or when the diagnostic variant mask asks for it.
 #pragma once
 
 #include "internal.h"
