@@ -85,10 +85,12 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 2-D bf16 tensor map over a row-major [outer, inner] array with 128-byte swizzle
-// (or none, for the epilogue's 32 x 32 store boxes).
+// 2-D bf16 tensor map over a row-major [outer, inner] array; 128-byte swizzle for
+// the GEMM operand tiles, 64-byte swizzle for the dz epilogue's 32 x 32 store boxes
+// (64-byte rows).
 bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
-              uint32_t box_inner, uint32_t box_outer, bool swizzle = true) {
+              uint32_t box_inner, uint32_t box_outer,
+              CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   auto fn = encode_fn();
   if (fn == nullptr) return false;
   cuuint64_t dims[2] = {inner, outer};
@@ -97,7 +99,7 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, 
   cuuint32_t es[2] = {1, 1};
   const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
                         strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                        swizzle,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -314,7 +316,7 @@ dpo_status backward_core(const Plan& p, const dpo_batch* batch, const float* lse
       uint16_t* G = reinterpret_cast<uint16_t*>(w + p.off_G);
       const uint16_t* hp0 = Hp + static_cast<size_t>(tok0) * p.d;
       CUtensorMap mHk, mWk, mGk, mWmn, mGmn, mHmn, mGst;
-      if (!make_map(&mGst, G, p.V, mc, 2ull * p.ldG, 32, 32, false) ||
+      if (!make_map(&mGst, G, p.V, mc, 2ull * p.ldG, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B) ||
           !make_map(&mHk, hp0, p.d, mc, 2ull * p.d, kBK, kBoxRows) ||
           !make_map(&mWk, batch->W, p.d, p.V, 2ull * p.d, kBK, kBoxRows) ||
           !make_map(&mGk, G, p.V, mc, 2ull * p.ldG, kBK, kBoxRows) ||

@@ -24,8 +24,9 @@ constexpr float kLog2eB = 1.4426950408889634f;
 
 // ------------------------------------------------------------------ dz epilogue
 // Each thread forms its row's 32 bf16 values of a chunk; the warp stages its 32 x 32
-// block in shared memory and one lane stores it with a TMA bulk tensor store (rows
-// beyond the chunk and columns beyond V fall outside the tensor map and are skipped).
+// block in shared memory (64-byte swizzled, matching the store map) and one lane
+// stores it with a TMA bulk tensor store (rows beyond the chunk and columns beyond V
+// fall outside the tensor map and are skipped).
 // Two staging buffers per warp: a buffer is refilled only after the store issued
 // from it two chunks earlier has finished reading it.
 struct EpiGrad {
@@ -74,10 +75,14 @@ struct EpiGrad {
     const uint32_t buf = ctx.stage + (c & 1) * (kEpiWarpBytes / 2);
     if (ctx.lane == 0) bulk_wait_group_read<1>();   // the store from this buffer is done
     __syncwarp();
-    const uint32_t dst = buf + ctx.lane * 64;       // row `lane`: 32 bf16 = 64 bytes
+    // row `lane`: 32 bf16 = 64 bytes, its four 16-byte pieces placed by the store
+    // map's 64-byte swizzle (piece q at q ^ ((row >> 1) & 3)), so the 32 lanes' stores
+    // spread over all 32 banks; the TMA store writes the rows back unswizzled
+    const uint32_t dst = buf + ctx.lane * 64;
+    const uint32_t sw = (ctx.lane >> 1) & 3;
 #pragma unroll
     for (int q = 0; q < 4; ++q)
-      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst + 16 * q),
+      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst + 16 * (q ^ sw)),
                    "r"(packed[4 * q]), "r"(packed[4 * q + 1]), "r"(packed[4 * q + 2]),
                    "r"(packed[4 * q + 3])
                    : "memory");
