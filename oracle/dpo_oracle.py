@@ -152,7 +152,7 @@ def sigmoid(x):
 
 
 def dpo_loss(pol, ref, beta, layout="halves", grad_scale=1.0, completion_len=None,
-             normalize=False, nll_weight=0.0):
+             normalize=False, nll_weight=0.0, pairs_total=None, nll_tokens_total=None):
     """Sigmoid DPO loss and its metrics, from policy and reference sequence sums.
 
     pol, ref: [2B] sequence log-prob sums in the row layout. The log-ratios are
@@ -168,6 +168,13 @@ def dpo_loss(pol, ref, beta, layout="halves", grad_scale=1.0, completion_len=Non
                   the chosen completions, read as the mean over all their tokens:
                   NLL = -(sum of chosen S_r) / (sum of chosen C_r), from raw sums.
     completion_len [2B] is needed by either variant.
+
+    Data-parallel shares ("Run Distributed Full-Model DPO with PyTorch FSDP", Step 1:
+    every rank holds part of the global batch): with pairs_total = B_g the batch
+    means (loss, accuracy, row_coef) divide by B_g instead of this call's B, and
+    with nll_tokens_total = N_g the NLL divides by N_g; the outputs are then this
+    part's share of the whole batch's values, and the shares of a partition of the
+    batch add up to the values of the whole.
     """
     pol = [float(x) for x in pol]
     ref = [float(x) for x in ref]
@@ -175,6 +182,7 @@ def dpo_loss(pol, ref, beta, layout="halves", grad_scale=1.0, completion_len=Non
     if R % 2:
         raise ValueError("odd number of rows")
     B = R // 2
+    Bdiv = B if pairs_total is None else int(pairs_total)
     C = None if completion_len is None else [int(c) for c in completion_len]
     if (normalize or nll_weight) and C is None:
         raise ValueError("completion lengths are needed for the loss variants")
@@ -196,13 +204,13 @@ def dpo_loss(pol, ref, beta, layout="halves", grad_scale=1.0, completion_len=Non
         w.append(wi)
         losses.append(softplus(-m))          # -log sigmoid(m)
         # d softplus(-m)/dm = -sigmoid(-m); dm/dpol[c] = beta, dm/dpol[r] = -beta
-        coef[c] = -grad_scale * beta * wi / B * scale[c]
-        coef[r] = +grad_scale * beta * wi / B * scale[r]
-    loss = math.fsum(losses) / B
+        coef[c] = -grad_scale * beta * wi / Bdiv * scale[c]
+        coef[r] = +grad_scale * beta * wi / Bdiv * scale[r]
+    loss = math.fsum(losses) / Bdiv
     nll = 0.0
     if nll_weight:
         chosen = [c for c, _ in pair_rows(B, layout)]
-        ntok = sum(C[c] for c in chosen)
+        ntok = sum(C[c] for c in chosen) if nll_tokens_total is None else int(nll_tokens_total)
         if ntok > 0:
             nll = -math.fsum(pol[c] for c in chosen) / ntok
             for c in chosen:
@@ -210,7 +218,7 @@ def dpo_loss(pol, ref, beta, layout="halves", grad_scale=1.0, completion_len=Non
         loss = loss + nll_weight * nll
     return {
         "loss": loss,
-        "accuracy": sum(1.0 for m in margins if m > 0) / B,
+        "accuracy": sum(1.0 for m in margins if m > 0) / Bdiv,
         "margins": np.array(margins),
         "chosen_rewards": np.array(rc),
         "rejected_rewards": np.array(rr),

@@ -373,6 +373,36 @@ def test_variant_row_coef_by_finite_differences(normalize, nll):
             assert out["row_coef"][r] == pytest.approx(fd, rel=1e-6, abs=1e-12)
 
 
+@pytest.mark.parametrize("normalize,nll", [(False, 0.0), (True, 0.0), (False, 0.6), (True, 0.4)])
+def test_data_parallel_shares_add_up_to_the_whole_batch(normalize, nll):
+    """Shares of a partition of the pairs into unequal parts (1, 2 and 4 pairs), each
+    computed with the whole batch's pair and chosen-token counts, add up to the loss,
+    accuracy and NLL of the whole batch; the row coefficients of each part are the
+    whole batch's coefficients of its rows, and per-pair values are unchanged."""
+    rng = np.random.default_rng(35)
+    B = 7
+    C = rng.integers(1, 30, 2 * B)
+    pol = -rng.uniform(0.5, 4, 2 * B) * C
+    ref = pol + rng.normal(0, 3, 2 * B)
+    kw = dict(completion_len=C, normalize=normalize, nll_weight=nll)
+    whole = O.dpo_loss(pol, ref, 0.1, "adjacent", grad_scale=0.5, **kw)
+    Ng = int(sum(C[0::2]))
+    tot = {"loss": 0.0, "accuracy": 0.0, "nll": 0.0}
+    for pairs in ([0], [1, 2], [3, 4, 5, 6]):
+        rows = np.array([r for i in pairs for r in (2 * i, 2 * i + 1)])
+        part = O.dpo_loss(pol[rows], ref[rows], 0.1, "adjacent", grad_scale=0.5,
+                          completion_len=C[rows], normalize=normalize, nll_weight=nll,
+                          pairs_total=B, nll_tokens_total=Ng)
+        for k in tot:
+            tot[k] += part[k]
+        np.testing.assert_allclose(part["row_coef"], whole["row_coef"][rows], rtol=1e-14,
+                                   atol=1e-17)
+        np.testing.assert_allclose(part["margins"], whole["margins"][pairs], rtol=1e-15)
+        np.testing.assert_allclose(part["weights"], whole["weights"][pairs], rtol=1e-15)
+    for k in tot:
+        assert tot[k] == pytest.approx(whole[k], rel=1e-13, abs=1e-15)
+
+
 # ---------------------------------------------------------------- logits-mean metrics
 def test_logits_mean_equal_vocab_rows_closed_form():
     """Every vocabulary row equal to w makes every logit of position t equal h_t . w,
