@@ -9,8 +9,12 @@ of the loss, the exchange a data-parallel optimiser step needs.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-Rank 0 prints one JSON line. The value is scored completion tokens per second
-over all ranks (max time over ranks, CUDA events, inputs resident in HBM).
+With --gpus N > 1 and no torchrun environment, the script starts its own N ranks
+(torch.distributed.run on this node) and runs inside them. Rank 0 prints one JSON
+line. The value is scored completion tokens per second over all ranks (max time
+over ranks, CUDA events, inputs resident in HBM); the K-step loop is timed --reps
+times and the median repetition is reported, with the spread and each repetition's
+SM clock.
 """
 from __future__ import annotations
 
@@ -55,6 +59,26 @@ def dist_env():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     return ws, rank, local
+
+
+def _free_port():
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def launch_ranks(argv, n):
+    """Re-run this script as n local ranks under torch.distributed.run (one process per
+    GPU); returns the launcher's exit status. NCCL's init log stays on (INFO) so a
+    scaling record shows the communicator's ranks, unless NCCL_DEBUG is already set."""
+    env = dict(os.environ)
+    env.setdefault("NCCL_DEBUG", "INFO")
+    env.setdefault("NCCL_DEBUG_SUBSYS", "INIT")
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr=127.0.0.1", f"--master-port={_free_port()}",
+           os.path.abspath(__file__), *argv]
+    return subprocess.run(cmd, env=env).returncode
 
 
 def rank_workload(name, rank, weights=True):
@@ -248,7 +272,7 @@ def run_reference(args):
     if rank != 0:
         return 0
     w = WL.make_config(args.workload)
-    s = OracleSample(w, per_row=args.ref_tokens_per_row)
+    s = OracleSample(w, per_row=args.cpu_tokens_per_row)
     for _ in range(args.warmup):
         s.step()
     t0 = time.perf_counter()
@@ -258,10 +282,10 @@ def run_reference(args):
     value = s.n_tokens * args.steps / dt
     cores = blas_threads()
     sample = (f"oracle fp64 (numpy/OpenBLAS) on one pair of the {args.workload} workload, "
-              f"completions cut to {args.ref_tokens_per_row} tokens per row ({s.n_tokens} tokens/step), "
+              f"completions cut to {args.cpu_tokens_per_row} tokens per row ({s.n_tokens} tokens/step), "
               f"full d and V; policy fwd + reference fwd + loss + backward")
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": max(ws, args.gpus),
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": {"workload": args.workload, "text": CONFIG_TEXT},
@@ -343,7 +367,14 @@ def run_ours(args):
              ("coef", 2 * B)]}
     stream = torch.cuda.current_stream(dev)
     sp = stream.cuda_stream
-    grad_scale = DP.grad_scale(ws_n)         # loss is the mean over the global batch
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    # data parallel: the loss is the mean over the whole batch of every rank. Each rank's
+    # loss call gets the whole batch's pair count, so its loss, accuracy and row
+    # coefficients are its share; one all-reduce sums the shares, the bucketed backward
+    # sums dW.
+    pairs_total = DP.global_counts(B, 0, device=dev)[0] if ws_n > 1 else 0
+    shares = torch.empty(2, device=dev)
+    outs["loss"], outs["accuracy"] = shares[0:1], shares[1:2]
 
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
 
@@ -368,17 +399,23 @@ def run_ours(args):
         libdpo.seq_logprobs(br, False, ref, None, None, ws, stream=sp)
         if timed is not None:
             ev[2].record(stream)
-        libdpo.loss(B, w.layout, pol, ref, w.beta, grad_scale, outs["loss"], outs["accuracy"],
-                    outs["margins"], outs["cr"], outs["rr"], outs["w"], outs["coef"], stream=sp)
+        libdpo.loss_ex(B, w.layout, pol, ref, w.beta, 1.0, outs["loss"], outs["accuracy"],
+                       outs["margins"], outs["cr"], outs["rr"], outs["w"], outs["coef"],
+                       pairs_total=pairs_total, stream=sp)
         if timed is not None:
             ev[3].record(stream)
-        libdpo.backward(bp, lse, outs["coef"], dH, dW, False, ws, stream=sp)
+        if ws_n > 1:
+            works = DP.backward_exchange(bp, lse, outs["coef"], dH, dW, ws,
+                                         n_buckets=args.dw_buckets,
+                                         max_sms=max(2, sms - args.comm_sms))
+            DP.finish(works)
+            DP.allreduce_shares(shares)
+        else:
+            libdpo.backward(bp, lse, outs["coef"], dH, dW, False, ws, stream=sp)
         if timed is not None:
             ev[4].record(stream)
             torch.cuda.synchronize(dev)
             timed.append([ev[i].elapsed_time(ev[i + 1]) for i in range(4)])
-        if ws_n > 1 and not fwd_only:
-            DP.allreduce_step(dW, outs["loss"])
 
     # launches of our kernels per step: upload + prep + GEMM + combine + rowsum per forward,
     # one loss kernel; the backward (one token chunk: the workspace holds all Nc rows of
@@ -387,7 +424,10 @@ def run_ours(args):
     uploads = math.ceil(w.R / 1024)
     fwd_launches = uploads + 4
     dh_launches = math.ceil(w.V / DH_VOCAB_CHUNK) if w.V >= 4 * DH_VOCAB_CHUNK else 1
-    bwd_launches = uploads + 3 + dh_launches
+    if ws_n > 1:   # dz, then dW by blocks of vocabulary rows, then dH
+        bwd_launches = uploads + 2 + len(DP.vocab_buckets(w.V, args.dw_buckets)) + dh_launches
+    else:
+        bwd_launches = uploads + 3 + dh_launches
     launches_per_step = (fwd_launches if fwd_only else 2 * fwd_launches + 1 + bwd_launches)
 
     for _ in range(args.warmup):
@@ -402,23 +442,27 @@ def run_ours(args):
         step(timed=breakdown)
     bd = np.median(np.array(breakdown), axis=0)
 
-    clocks = ClockSampler(local)
-    if ws_n > 1:
-        dist.barrier()
-    torch.cuda.synchronize(dev)
-    clocks.start()
-    time.sleep(0.3)
-    t_start = torch.cuda.Event(enable_timing=True)
-    t_end = torch.cuda.Event(enable_timing=True)
-    t_start.record(stream)
-    for _ in range(args.steps):
-        step()
-    t_end.record(stream)
-    torch.cuda.synchronize(dev)
-    if ws_n > 1:
-        dist.barrier()
-    clk = clocks.stop()
-    ms = t_start.elapsed_time(t_end)
+    # the K-step loop, timed args.reps times: barrier + synchronize on both sides of each
+    # repetition, CUDA events on the launching stream, clocks sampled during each one
+    rep_ms, rep_clk = [], []
+    for _ in range(args.reps):
+        clocks = ClockSampler(local)
+        if ws_n > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        clocks.start()
+        time.sleep(0.3)
+        t_start = torch.cuda.Event(enable_timing=True)
+        t_end = torch.cuda.Event(enable_timing=True)
+        t_start.record(stream)
+        for _ in range(args.steps):
+            step()
+        t_end.record(stream)
+        torch.cuda.synchronize(dev)
+        if ws_n > 1:
+            dist.barrier()
+        rep_clk.append(clocks.stop())
+        rep_ms.append(t_start.elapsed_time(t_end))
     st = libdpo.check(sp)
     if st != libdpo.OK:
         raise RuntimeError(f"device status after timing: {libdpo.status_string(st)}")
@@ -457,29 +501,32 @@ def run_ours(args):
 
     for i in range(2):
         consumed[i].record(stream)
-    if ws_n > 1:
-        dist.barrier()
-    torch.cuda.synchronize(dev)
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    upload(0)
-    for i in range(e2e_steps):
-        if i + 1 < e2e_steps:
-            upload(i + 1)
-        stream.wait_event(uploaded[i % 2])
-        bp_i, br_i = batches[i % 2]
-        step_with(bp_i, br_i)
-        consumed[i % 2].record(stream)
-        if fwd_only:
-            res_dev = pol
-        else:
-            res_dev = torch.cat([outs["loss"], outs["accuracy"], outs["margins"], outs["cr"], outs["rr"]])
-        res_host[:res_dev.numel()].copy_(res_dev, non_blocking=True)
-        stream.synchronize()                                 # the host reads the step's result
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    e2e_ms = e0.elapsed_time(e1)
+    e2e_reps = []
+    for _ in range(args.reps):
+        if ws_n > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        upload(0)
+        for i in range(e2e_steps):
+            if i + 1 < e2e_steps:
+                upload(i + 1)
+            stream.wait_event(uploaded[i % 2])
+            bp_i, br_i = batches[i % 2]
+            step_with(bp_i, br_i)
+            consumed[i % 2].record(stream)
+            if fwd_only:
+                res_dev = pol
+            else:
+                res_dev = torch.cat([outs["loss"], outs["accuracy"], outs["margins"], outs["cr"],
+                                     outs["rr"]])
+            res_host[:res_dev.numel()].copy_(res_dev, non_blocking=True)
+            stream.synchronize()                             # the host reads the step's result
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_reps.append(e0.elapsed_time(e1))
     h2d = H_host.numel() * 2 + tok_host.numel() * 4
     d2h = (w.R if fwd_only else 2 + 3 * B) * 4
 
@@ -506,16 +553,26 @@ def run_ours(args):
         cublas = cublas_sustained(torch, dev, stream, seconds=1.5)
 
     # ------------------------------------------------------------ aggregate over ranks
-    t = torch.tensor([ms, e2e_ms, float(Nc)], device=dev, dtype=torch.float64)
+    # each repetition's time is the max over ranks; the median repetition is reported
+    t = torch.tensor(rep_ms + e2e_reps + [float(Nc)], device=dev, dtype=torch.float64)
     if ws_n > 1:
         tmax = t.clone()
         dist.all_reduce(tmax, op=dist.ReduceOp.MAX)
         tsum = t.clone()
         dist.all_reduce(tsum, op=dist.ReduceOp.SUM)
-        ms, e2e_ms = float(tmax[0]), float(tmax[1])
-        total_nc = float(tsum[2])
+        rep_ms = [float(x) for x in tmax[:args.reps]]
+        e2e_reps = [float(x) for x in tmax[args.reps:2 * args.reps]]
+        total_nc = float(tsum[-1])
     else:
         total_nc = float(Nc)
+    order = sorted(range(args.reps), key=lambda i: rep_ms[i])
+    med = order[(args.reps - 1) // 2]                 # the median repetition (lower middle)
+    ms = rep_ms[med]
+    clk = dict(rep_clk[med]) if rep_clk[med] else None
+    if clk is not None:        # throttle reasons seen in any repetition
+        clk["reasons"] = sorted({r for c in rep_clk if c for r in c["reasons"]})
+    e2e_ms = sorted(e2e_reps)[(args.reps - 1) // 2]
+    rep_mhz = [c["sm_mhz"] if c else None for c in rep_clk]
 
     peaks, peak_src = load_peaks()
     value = total_nc * args.steps / (ms / 1e3)
@@ -542,7 +599,7 @@ def run_ours(args):
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded; random-init LM-head weights of the Llama-3.1-8B head shape)",
             "config": {"workload": args.workload, "text": CONFIG_TEXT, "rows_per_gpu": w.R,
-                       "gemm_single_cta_mask": args.gemm_variant,
+                       "gemm_variant_mask": args.gemm_variant,
                        "pairs_per_gpu": B, "seq_len": w.L, "d": w.d, "V": w.V,
                        "scored_tokens_per_gpu": Nc, "global_batch_pairs": B * ws_n,
                        "parallelism": f"dp{ws_n}",
@@ -565,6 +622,16 @@ def run_ours(args):
                     "d2h_bytes_per_step": d2h, "steps": e2e_steps},
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clk,
+            "repeats": {
+                "n": args.reps, "reported": "median repetition",
+                "ms_per_step": [x / args.steps for x in rep_ms],
+                "sm_mhz": rep_mhz,
+                "spread_pct": 100.0 * (max(rep_ms) - min(rep_ms)) / ms,
+                "ms_x_ghz_per_step": [x / args.steps * m / 1e3 if m else None
+                                      for x, m in zip(rep_ms, rep_mhz)],
+                "e2e_ms_per_step": [x / e2e_steps for x in e2e_reps],
+                "reasons": sorted({r for c in rep_clk if c for r in c["reasons"]}),
+            },
             "cpu_baseline": cpu,
             "cublas_same_box": cublas,
             "logits_mean_metric": {"ms": lm_ms, "bytes": lm_bytes,
@@ -591,13 +658,29 @@ def main(argv=None):
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(WL.CONFIGS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-cublas-reference", action="store_true")
-    ap.add_argument("--gemm-variant", type=int, default=0, choices=range(16),
-                    help="mask, one bit per GEMM (forward, dz, dH, dW): set = single-CTA kernel")
-    ap.add_argument("--cpu-tokens-per-row", type=int, default=64)
-    ap.add_argument("--ref-tokens-per-row", type=int, default=4)
-    args = ap.parse_args(argv)
+    ap.add_argument("--gemm-variant", type=int, default=0, choices=range(256),
+                    help="mask, per GEMM (forward, dz, dH, dW) bit k: single-CTA kernel, "
+                         "bit 4 + k: static tile schedule")
+    ap.add_argument("--cpu-tokens-per-row", type=int, default=64,
+                    help="oracle sample (CPU baseline and reference arm): completion tokens "
+                         "per row of one pair")
+    ap.add_argument("--reps", type=int, default=5,
+                    help="repetitions of the timed K-step loop (the median is reported)")
+    ap.add_argument("--dw-buckets", type=int, default=8,
+                    help="data parallel: blocks of dW rows whose all-reduce overlaps the next")
+    ap.add_argument("--comm-sms", type=int, default=16,
+                    help="data parallel: SMs the backward GEMMs leave free for NCCL")
+    raw = sys.argv[1:] if argv is None else list(argv)
+    args = ap.parse_args(raw)
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
+    args.reps = max(1, args.reps)
+    ws = int(os.environ.get("WORLD_SIZE", "0"))
+    if ws == 0 and args.gpus > 1:
+        return launch_ranks(raw, args.gpus)
+    if ws > 0 and ws != args.gpus:
+        print(f"bench.py: WORLD_SIZE={ws} but --gpus {args.gpus}", file=sys.stderr)
+        return 2
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

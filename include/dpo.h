@@ -143,11 +143,23 @@ dpo_status dpo_loss(int32_t B, int32_t layout, const float* pol, const float* re
  *                   policy sums) / (their total completion length), i.e. the mean
  *                   over all chosen completion tokens
  *   completion_len  device [2B] int32 C_r in the row layout; required when
- *                   normalize != 0 or nll_weight > 0, else may be NULL */
+ *                   normalize != 0 or nll_weight > 0, else may be NULL
+ *   pairs_total     data parallelism: when > 0 the batch means (loss, accuracy,
+ *                   row_coef) divide by B_g = pairs_total, the pair count summed over
+ *                   every rank, instead of this call's B (B_g < B is refused)
+ *   nll_tokens_total  when > 0 the NLL divides by N_g, the chosen completion tokens
+ *                   summed over every rank, instead of this call's own count
+ * With both set, loss, accuracy, nll and row_coef are this rank's share of the
+ * whole batch's values: summing them over the ranks (one all-reduce) gives the
+ * single-process result on the whole batch, for unequal shards too ("Run
+ * Distributed Full-Model DPO with PyTorch FSDP", Step 1: every rank holds part of
+ * the global batch). Margins, rewards and weights are per pair and unchanged. */
 typedef struct {
   int32_t normalize;
   float nll_weight;
   const int32_t* completion_len;
+  int32_t pairs_total;      /* 0, or B_g >= B: the pairs of the whole data-parallel batch */
+  int64_t nll_tokens_total; /* 0, or N_g >= 0: the whole batch's chosen completion tokens */
 } dpo_loss_options;
 
 /* dpo_loss with the variants above (opt may be NULL: then it equals dpo_loss).
@@ -167,10 +179,38 @@ dpo_status dpo_loss_ex(int32_t B, int32_t layout, const float* pol, const float*
  *               accumulate_dW != 0 (gradient accumulation over micro-batches)
  *   ws          device workspace, >= bwd_min_bytes, 256-byte aligned
  * with dz[t, v] = row_coef[r(t)] * (1[v = tokens[r, t+1]] - softmax(z_t)[v]). The
- * logits are recomputed tile by tile. dH may be NULL (only dW is formed). */
+ * logits are recomputed tile by tile. dH may be NULL (only dW is formed).
+ * dW may be NULL too: then the whole batch must fit one workspace chunk (ws_bytes >=
+ * bwd_bytes and Nc <= 2^20, else DPO_ERR_WORKSPACE) and the logit gradient dz stays
+ * in the workspace, where dpo_backward_dw and dpo_backward_dh read it. */
 dpo_status dpo_backward(const dpo_batch* batch, const float* lse_state, const float* row_coef,
                         float* dH, float* dW, int accumulate_dW, void* ws, size_t ws_bytes,
                         void* stream);
+
+/* Rows [v_begin, v_end) of dW from the dz that a preceding dpo_backward(dW = NULL) on
+ * the same batch left in ws (ws unchanged since). Splitting dW by vocabulary rows
+ * lets a data-parallel caller start the all-reduce of each finished block of rows
+ * while the next block is computed ("Run Distributed Full-Model DPO with PyTorch
+ * FSDP", Step 1: the ranks' gradients are summed).
+ *   v_begin, v_end  0 <= v_begin <= v_end <= V; v_begin a multiple of 8, v_end a
+ *                   multiple of 8 or V
+ *   dW              device [V, d] fp32, the whole array: only the range's rows are
+ *                   written (or accumulated when accumulate_dW != 0)
+ *   max_sms         0: use every SM; > 0: at most that many, leaving the others free
+ *                   for kernels of other streams (a collective) to run beside it
+ * Every row is computed with the same order of operations as in dpo_backward, so the
+ * result does not depend on the split or on max_sms. Errors: DPO_ERR_INVALID_ARG for
+ * a bad range, NULL dW or max_sms < 0; DPO_ERR_WORKSPACE when ws cannot hold the whole
+ * batch's dz. */
+dpo_status dpo_backward_dw(const dpo_batch* batch, int32_t v_begin, int32_t v_end, float* dW,
+                           int accumulate_dW, int32_t max_sms, void* ws, size_t ws_bytes,
+                           void* stream);
+
+/* dH (device [R, L, d] fp32, fully written, 0 at unscored positions) from the dz a
+ * preceding dpo_backward(dW = NULL) left in ws; max_sms and errors as for
+ * dpo_backward_dw. The same values as dpo_backward's dH. */
+dpo_status dpo_backward_dh(const dpo_batch* batch, float* dH, int32_t max_sms, void* ws,
+                           size_t ws_bytes, void* stream);
 
 /* ---- Vocabulary-parallel head ----------------------------------------------
  * W split by vocabulary rows across ranks, every rank holding the same batch (the
@@ -259,7 +299,8 @@ dpo_status dpo_logits_mean(const dpo_batch* batch, int32_t layout, float* means,
  *   whose forward workspace (dpo_workspace_size's fwd_bytes) exceeds that size is
  *   refused with DPO_ERR_WORKSPACE before any device work.
  *   Set-up: the first call on a device, made with that device current, looks the
- *   array's address up (cudaGetSymbolAddress); make that first call before any
+ *   array's address up (cudaGetSymbolAddress), as does the first call after that
+ *   device's context was destroyed and rebuilt; make that first call before any
  *   stream capture.
  *   Sharing: all calls on a device use the same array and it keeps the last
  *   call's contents (every byte a call reads is written by that call first).
@@ -299,13 +340,18 @@ dpo_status dpo_fingerprint(const void* data, size_t bytes, uint64_t* out, void* 
 dpo_status dpo_selftest_wait_timeout(uint32_t budget_ms, void* stream);
 
 /* Which tensor-core GEMM kernel later calls of this process use, as a mask with
- * one bit per GEMM: bit 0 the forward (logits + log-sum-exp), bit 1 the backward's
- * logit recompute (dz), bit 2 dH = dz.W, bit 3 dW = dz^T.H. A clear bit runs that
- * GEMM on a pair of CTAs (tcgen05.mma.cta_group::2, 256 x 256 tiles) when the
- * device can co-schedule CTA pairs, unless one CTA per 128 x 256 tile fills the
- * GPU's waves more than 5 % better for that launch's shape; a set bit always runs
- * it on one CTA. Both give the same results within rounding. Default 0. Returns
- * the previous mask, or -1 for a value outside 0..15. */
+ * two bits per GEMM k: k = 0 the forward (logits + log-sum-exp), 1 the backward's
+ * logit recompute (dz), 2 dH = dz.W, 3 dW = dz^T.H.
+ *   bit k      clear: the GEMM runs on pairs of CTAs (tcgen05.mma.cta_group::2,
+ *              256 x 256 tiles) when the device can co-schedule CTA pairs, unless one
+ *              CTA per 128 x 256 tile fills the GPU's waves more than 5 % better for
+ *              that launch's shape; set: always on one CTA per tile.
+ *   bit 4 + k  clear: the CTA pairs claim tiles in raster order from a counter in the
+ *              workspace (the tiles in flight stay one contiguous window of the
+ *              raster); set: static round-robin (pair p takes tiles p, p + pairs, ...).
+ * Every choice gives the same results (each tile is computed the same way). Default
+ * 0. Returns the previous mask, or -1 for a value outside 0..255. A diagnostic for
+ * measurements; the default is the fastest measured. */
 int32_t dpo_set_gemm_variant(int32_t variant);
 
 /* Static description of a status code. */

@@ -39,6 +39,7 @@ std::atomic<int> g_gemm_variant{0};
 
 struct DevInfo {
   bool ready = false;
+  void* ctx = nullptr;     // the context the cached addresses belong to
   int* status = nullptr;
   int sms = 0;
 };
@@ -48,9 +49,12 @@ DevInfo g_dev[256];
 dpo_status device_info(DevInfo* out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 256) return DPO_ERR_CUDA;
+  void* ctx = nullptr;
+  if (!dpo::current_context(&ctx)) return DPO_ERR_CUDA;
   std::lock_guard<std::mutex> lk(g_mu);
   DevInfo& di = g_dev[dev];
-  if (!di.ready) {
+  if (!di.ready || di.ctx != ctx) {     // first call, or the context was rebuilt
+    di.ready = false;
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_dpo_status_word) != cudaSuccess) return DPO_ERR_CUDA;
     int sms = 0;
@@ -58,6 +62,7 @@ dpo_status device_info(DevInfo* out) {
       return DPO_ERR_CUDA;
     di.status = static_cast<int*>(p);
     di.sms = sms;
+    di.ctx = ctx;
     di.ready = true;
   }
   *out = di;
@@ -273,27 +278,90 @@ dpo_status forward_core(const Plan& p, const dpo_batch* batch, void* ws, float* 
   return cuda_status(launch_combine(part, p.ldp, p.S, zy, sc.y, p.Nc, lp, lse_out, zy_out, st));
 }
 
+// SMs a launch may use: all of them, or at most max_sms (> 0) to leave the rest to
+// kernels that run beside it (a collective on another stream).
+int sm_budget(const DevInfo& di, int max_sms) {
+  return max_sms > 0 && max_sms < di.sms ? max_sms : di.sms;
+}
+
+// Token chunk of the backward that fits the workspace (a multiple of 128 unless it
+// covers every scored position; never more than kMaxAccumK, dW's K per chunk).
+int backward_chunk(const Plan& p, size_t ws_bytes) {
+  const size_t rows_fit = ws_bytes > p.off_G ? (ws_bytes - p.off_G) / p.g_row_bytes : 0;
+  int Mc = static_cast<int>(std::min<size_t>(rows_fit, static_cast<size_t>(p.Nc)));
+  Mc = std::min(Mc, kMaxAccumK);
+  if (Mc < p.Nc) Mc = Mc / kMinChunk * kMinChunk;
+  return Mc;
+}
+
+// dH rows of the packed positions [tok0, tok0 + mc) from the dz chunk in the workspace:
+// dH = dz . W, reduced over the vocabulary in one launch or in chunks of kDhVocabChunk
+// columns for a long vocabulary (never longer than kMaxAccumK), the later chunks added
+// to the rows by the epilogue.
+dpo_status run_dh(const Plan& p, const dpo_batch* batch, uint8_t* w, const Sched& sc, int tok0,
+                  int mc, float* dH, int sms, const DevCtl& ctl, cudaStream_t st) {
+  if (p.dtype != DPO_BF16) {
+    const float* G = reinterpret_cast<const float*>(w + p.off_G);
+    return cuda_status(launch_f32_dh(G, static_cast<const float*>(batch->W), sc, tok0, mc, p.d,
+                                     p.V, dH, st));
+  }
+  const uint16_t* G = reinterpret_cast<const uint16_t*>(w + p.off_G);
+  const int dh_chunk = p.V >= kDhChunkFrom ? kDhVocabChunk : kMaxAccumK;
+  for (int v0 = 0; v0 < p.V; v0 += dh_chunk) {
+    const int vc = std::min(dh_chunk, p.V - v0);
+    CUtensorMap mGk, mWmn;
+    if (!make_map(&mGk, G + v0, vc, mc, 2ull * p.ldG, kBK, kBoxRows) ||
+        !make_map(&mWmn, static_cast<const uint16_t*>(batch->W) + static_cast<size_t>(v0) * p.d,
+                  p.d, vc, 2ull * p.d, kBoxMN, kBK))
+      return DPO_ERR_CUDA;
+    if (launch_bwd_dh(mGk, mWmn, mc, vc, p.d, tok0, sc.dst, dH, v0 > 0 ? 1 : 0, sms, sc.sync, ctl,
+                      st) != cudaSuccess)
+      return DPO_ERR_CUDA;
+  }
+  return DPO_OK;
+}
+
+// dW rows [v0, v1) (+)= dz^T . Hp for the packed positions [tok0, tok0 + mc) of the dz
+// chunk in the workspace; dW points at the whole [V, d] array.
+dpo_status run_dw(const Plan& p, const dpo_batch* batch, uint8_t* w, const Sched& sc, int tok0,
+                  int mc, int v0, int v1, float* dW, int acc, int sms, const DevCtl& ctl,
+                  cudaStream_t st) {
+  if (v1 <= v0) return DPO_OK;
+  if (p.dtype != DPO_BF16) {
+    const float* G = reinterpret_cast<const float*>(w + p.off_G);
+    return cuda_status(launch_f32_dw(G, static_cast<const float*>(batch->H), sc, tok0, mc, p.d,
+                                     p.V, v0, v1, dW, acc, st));
+  }
+  const uint16_t* G = reinterpret_cast<const uint16_t*>(w + p.off_G);
+  const uint16_t* hp0 = reinterpret_cast<const uint16_t*>(w + p.off_hp) +
+                        static_cast<size_t>(tok0) * p.d;
+  CUtensorMap mGmn, mHmn;
+  if (!make_map(&mGmn, G + v0, v1 - v0, mc, 2ull * p.ldG, kBoxMN, kBK) ||
+      !make_map(&mHmn, hp0, p.d, mc, 2ull * p.d, kBoxMN, kBK))
+    return DPO_ERR_CUDA;
+  return cuda_status(launch_bwd_dw(mGmn, mHmn, mc, v1 - v0, p.d,
+                                   dW + static_cast<size_t>(v0) * p.d, acc, sms, sc.sync, ctl,
+                                   st));
+}
+
 // Backward of sum_r row_coef[r] S_r for this call's vocabulary rows: dz chunks,
-// dH (fully written) and dW (written or accumulated).
+// dH (fully written, when dH != NULL) and dW (written or accumulated, when dW != NULL).
+// With dW == NULL the whole batch must fit one chunk: its dz then stays in the
+// workspace for dpo_backward_dw / dpo_backward_dh.
 dpo_status backward_core(const Plan& p, const dpo_batch* batch, const float* lse_state,
                          const float* row_coef, float* dH, float* dW, int accumulate_dW, void* ws,
                          size_t ws_bytes, void* stream) {
   dpo_status s = DPO_OK;
-  if ((p.Nc > 0 && lse_state == nullptr) || row_coef == nullptr || dW == nullptr)
-    return DPO_ERR_INVALID_ARG;
+  if ((p.Nc > 0 && lse_state == nullptr) || row_coef == nullptr) return DPO_ERR_INVALID_ARG;
   if (!ws_ok(ws, ws_bytes, p.bwd_min)) return DPO_ERR_WORKSPACE;
+  const int Mc = backward_chunk(p, ws_bytes);
+  if (p.Nc > 0 && Mc < 1) return DPO_ERR_WORKSPACE;
+  if (dW == nullptr && Mc < p.Nc) return DPO_ERR_WORKSPACE;   // dz must stay whole
   DevInfo di;
   if ((s = device_info(&di)) != DPO_OK) return s;
   const DevCtl ctl = make_ctl(di);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t* w = static_cast<uint8_t*>(ws);
-
-  // Token chunk that fits the workspace (a multiple of 128 unless it covers all).
-  size_t rows_fit = (ws_bytes - p.off_G) / p.g_row_bytes;
-  int Mc = static_cast<int>(std::min<size_t>(rows_fit, static_cast<size_t>(p.Nc)));
-  Mc = std::min(Mc, kMaxAccumK);           // dW's K: positions per chunk
-  if (Mc < p.Nc) Mc = Mc / kMinChunk * kMinChunk;
-  if (p.Nc > 0 && Mc < 1) return DPO_ERR_WORKSPACE;
 
   if ((s = stage_schedule(p, batch, ws, ctl, st)) != DPO_OK) return s;
   const Sched sc = sched_of(p, ws);
@@ -302,70 +370,73 @@ dpo_status backward_core(const Plan& p, const dpo_batch* batch, const float* lse
           cudaSuccess)
     return DPO_ERR_CUDA;
   if (p.Nc == 0) {
-    if (!accumulate_dW &&
+    if (dW != nullptr && !accumulate_dW &&
         cudaMemsetAsync(dW, 0, sizeof(float) * static_cast<size_t>(p.V) * p.d, st) != cudaSuccess)
       return DPO_ERR_CUDA;
     return DPO_OK;
   }
   const bool bf16 = p.dtype == DPO_BF16;
-  const uint16_t* Hp = reinterpret_cast<const uint16_t*>(w + p.off_hp);
   for (int tok0 = 0; tok0 < p.Nc; tok0 += Mc) {
     const int mc = std::min(Mc, p.Nc - tok0);
     const int acc = (accumulate_dW || tok0 > 0) ? 1 : 0;
     if (bf16) {
       uint16_t* G = reinterpret_cast<uint16_t*>(w + p.off_G);
-      const uint16_t* hp0 = Hp + static_cast<size_t>(tok0) * p.d;
-      CUtensorMap mHk, mWk, mGk, mWmn, mGmn, mHmn, mGst;
+      const uint16_t* hp0 = reinterpret_cast<const uint16_t*>(w + p.off_hp) +
+                            static_cast<size_t>(tok0) * p.d;
+      CUtensorMap mHk, mWk, mGst;
       if (!make_map(&mGst, G, p.V, mc, 2ull * p.ldG, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B) ||
           !make_map(&mHk, hp0, p.d, mc, 2ull * p.d, kBK, kBoxRows) ||
-          !make_map(&mWk, batch->W, p.d, p.V, 2ull * p.d, kBK, kBoxRows) ||
-          !make_map(&mGk, G, p.V, mc, 2ull * p.ldG, kBK, kBoxRows) ||
-          !make_map(&mWmn, batch->W, p.d, p.V, 2ull * p.d, kBoxMN, kBK) ||
-          !make_map(&mGmn, G, p.V, mc, 2ull * p.ldG, kBoxMN, kBK) ||
-          !make_map(&mHmn, hp0, p.d, mc, 2ull * p.d, kBoxMN, kBK))
+          !make_map(&mWk, batch->W, p.d, p.V, 2ull * p.d, kBK, kBoxRows))
         return DPO_ERR_CUDA;
       if (launch_bwd_grad(mHk, mWk, mGst, mc, p.V, p.d, tok0, sc.y, lse_state, row_coef,
                           sc.rowid, di.sms, sc.sync, ctl, st) != cudaSuccess)
         return DPO_ERR_CUDA;
-      // dH = dz . W reduces over the vocabulary: one launch, or chunks of kDhVocabChunk
-      // columns for a long vocabulary (never longer than kMaxAccumK), the later ones
-      // added to the rows by the epilogue.
-      const int dh_chunk = p.V >= kDhChunkFrom ? kDhVocabChunk : kMaxAccumK;
-      for (int v0 = 0; dH != nullptr && v0 < p.V; v0 += dh_chunk) {
-        const int vc = std::min(dh_chunk, p.V - v0);
-        CUtensorMap mGkc = mGk, mWmnc = mWmn;
-        if (v0 > 0 || vc < p.V) {
-          if (!make_map(&mGkc, G + v0, vc, mc, 2ull * p.ldG, kBK, kBoxRows) ||
-              !make_map(&mWmnc, static_cast<const uint16_t*>(batch->W) + static_cast<size_t>(v0) * p.d,
-                        p.d, vc, 2ull * p.d, kBoxMN, kBK))
-            return DPO_ERR_CUDA;
-        }
-        if (launch_bwd_dh(mGkc, mWmnc, mc, vc, p.d, tok0, sc.dst, dH, v0 > 0 ? 1 : 0, di.sms,
-                          sc.sync, ctl, st) != cudaSuccess)
-          return DPO_ERR_CUDA;
-      }
-      if (launch_bwd_dw(mGmn, mHmn, mc, p.V, p.d, dW, acc, di.sms, sc.sync, ctl, st) !=
-          cudaSuccess)
-        return DPO_ERR_CUDA;
     } else {
-      float* G = reinterpret_cast<float*>(w + p.off_G);
-      const float* H = static_cast<const float*>(batch->H);
-      const float* W = static_cast<const float*>(batch->W);
-      if (launch_f32_grad(H, W, sc, tok0, mc, p.d, p.V, lse_state, row_coef, G, st) !=
-          cudaSuccess)
-        return DPO_ERR_CUDA;
-      if (dH != nullptr && launch_f32_dh(G, W, sc, tok0, mc, p.d, p.V, dH, st) != cudaSuccess)
-        return DPO_ERR_CUDA;
-      if (launch_f32_dw(G, H, sc, tok0, mc, p.d, p.V, dW, acc, st) != cudaSuccess)
+      if (launch_f32_grad(static_cast<const float*>(batch->H),
+                          static_cast<const float*>(batch->W), sc, tok0, mc, p.d, p.V, lse_state,
+                          row_coef, reinterpret_cast<float*>(w + p.off_G), st) != cudaSuccess)
         return DPO_ERR_CUDA;
     }
+    if (dH != nullptr && (s = run_dh(p, batch, w, sc, tok0, mc, dH, di.sms, ctl, st)) != DPO_OK)
+      return s;
+    if (dW != nullptr &&
+        (s = run_dw(p, batch, w, sc, tok0, mc, 0, p.V, dW, acc, di.sms, ctl, st)) != DPO_OK)
+      return s;
   }
+  return DPO_OK;
+}
+
+// Checks shared by the calls that continue from the dz a dpo_backward(dW = NULL) left
+// in the workspace: the whole batch in one chunk.
+dpo_status dz_resident(const Plan& p, const void* ws, size_t ws_bytes, int max_sms) {
+  if (max_sms < 0) return DPO_ERR_INVALID_ARG;
+  if (!ws_ok(ws, ws_bytes, p.bwd_min)) return DPO_ERR_WORKSPACE;
+  if (backward_chunk(p, ws_bytes) < p.Nc) return DPO_ERR_WORKSPACE;
   return DPO_OK;
 }
 
 }  // namespace
 
 int dpo::gemm_variant() { return g_gemm_variant.load(); }
+
+bool dpo::current_context(void** ctx) {
+  // The runtime's calls above made the device's primary context current; the driver's
+  // cuCtxGetCurrent (reached without linking libcuda) names it.
+  static PFN_cuCtxGetCurrent_v4000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+  });
+  if (fn == nullptr) return false;
+  CUcontext c = nullptr;
+  if (fn(&c) != CUDA_SUCCESS || c == nullptr) return false;
+  *ctx = c;
+  return true;
+}
 
 extern "C" {
 
@@ -459,8 +530,8 @@ dpo_status dpo_loss(int32_t B, int32_t layout, const float* pol, const float* re
   if (pol == nullptr || ref == nullptr || loss == nullptr) return DPO_ERR_INVALID_ARG;
   if (!(beta > 0.f) || !std::isfinite(beta) || !std::isfinite(grad_scale))
     return DPO_ERR_INVALID_ARG;
-  return cuda_status(launch_loss(B, layout, pol, ref, beta, grad_scale, 0, 0.0, nullptr, loss,
-                                 accuracy, margins, chosen_rewards, rejected_rewards, weights,
+  return cuda_status(launch_loss(B, layout, pol, ref, beta, grad_scale, 0, 0.0, nullptr, 0, 0,
+                                 loss, accuracy, margins, chosen_rewards, rejected_rewards, weights,
                                  row_coef, nullptr, static_cast<cudaStream_t>(stream)));
 }
 
@@ -477,15 +548,20 @@ dpo_status dpo_loss_ex(int32_t B, int32_t layout, const float* pol, const float*
   int normalize = 0;
   float nll_weight = 0.f;
   const int32_t* clen = nullptr;
+  long long pairs_total = 0, ntok_total = 0;
   if (opt != nullptr) {
     normalize = opt->normalize ? 1 : 0;
     nll_weight = opt->nll_weight;
     clen = opt->completion_len;
+    pairs_total = opt->pairs_total;
+    ntok_total = opt->nll_tokens_total;
     if (!std::isfinite(nll_weight) || nll_weight < 0.f) return DPO_ERR_INVALID_ARG;
     if ((normalize || nll_weight > 0.f) && clen == nullptr) return DPO_ERR_INVALID_ARG;
+    if (pairs_total != 0 && pairs_total < B) return DPO_ERR_INVALID_ARG;
+    if (ntok_total < 0) return DPO_ERR_INVALID_ARG;
   }
   return cuda_status(launch_loss(B, layout, pol, ref, beta, grad_scale, normalize, nll_weight,
-                                 clen, loss, accuracy, margins, chosen_rewards, rejected_rewards,
+                                 clen, pairs_total, ntok_total, loss, accuracy, margins, chosen_rewards, rejected_rewards,
                                  weights, row_coef, nll, static_cast<cudaStream_t>(stream)));
 }
 
@@ -497,6 +573,52 @@ dpo_status dpo_backward(const dpo_batch* batch, const float* lse_state, const fl
   const dpo_status s = make_plan(batch, &p);
   if (s != DPO_OK) return s;
   return backward_core(p, batch, lse_state, row_coef, dH, dW, accumulate_dW, ws, ws_bytes, stream);
+}
+
+dpo_status dpo_backward_dw(const dpo_batch* batch, int32_t v_begin, int32_t v_end, float* dW,
+                           int accumulate_dW, int32_t max_sms, void* ws, size_t ws_bytes,
+                           void* stream) {
+  NvtxRange nvtx_range("dpo_backward_dw");
+  Plan p;
+  dpo_status s = make_plan(batch, &p);
+  if (s != DPO_OK) return s;
+  if (dW == nullptr || v_begin < 0 || v_end > p.V || v_begin > v_end || v_begin % 8 != 0 ||
+      (v_end % 8 != 0 && v_end != p.V))
+    return DPO_ERR_INVALID_ARG;
+  if ((s = dz_resident(p, ws, ws_bytes, max_sms)) != DPO_OK) return s;
+  if (v_begin == v_end) return DPO_OK;
+  DevInfo di;
+  if ((s = device_info(&di)) != DPO_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (p.Nc == 0) {
+    if (!accumulate_dW &&
+        cudaMemsetAsync(dW + static_cast<size_t>(v_begin) * p.d, 0,
+                        sizeof(float) * static_cast<size_t>(v_end - v_begin) * p.d,
+                        st) != cudaSuccess)
+      return DPO_ERR_CUDA;
+    return DPO_OK;
+  }
+  return run_dw(p, batch, static_cast<uint8_t*>(ws), sched_of(p, ws), 0, p.Nc, v_begin, v_end, dW,
+                accumulate_dW ? 1 : 0, sm_budget(di, max_sms), make_ctl(di), st);
+}
+
+dpo_status dpo_backward_dh(const dpo_batch* batch, float* dH, int32_t max_sms, void* ws,
+                           size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_range("dpo_backward_dh");
+  Plan p;
+  dpo_status s = make_plan(batch, &p);
+  if (s != DPO_OK) return s;
+  if (dH == nullptr) return DPO_ERR_INVALID_ARG;
+  if ((s = dz_resident(p, ws, ws_bytes, max_sms)) != DPO_OK) return s;
+  DevInfo di;
+  if ((s = device_info(&di)) != DPO_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(dH, 0, sizeof(float) * static_cast<size_t>(p.R) * p.L * p.d, st) !=
+      cudaSuccess)
+    return DPO_ERR_CUDA;
+  if (p.Nc == 0) return DPO_OK;
+  return run_dh(p, batch, static_cast<uint8_t*>(ws), sched_of(p, ws), 0, p.Nc, dH,
+                sm_budget(di, max_sms), make_ctl(di), st);
 }
 
 dpo_status dpo_shard_backward(const dpo_batch* batch, const dpo_vocab_shard* shard,
@@ -566,7 +688,7 @@ dpo_status dpo_selftest_wait_timeout(uint32_t budget_ms, void* stream) {
 }
 
 int32_t dpo_set_gemm_variant(int32_t variant) {
-  if (variant < 0 || variant > 15) return -1;
+  if (variant < 0 || variant > 255) return -1;
   return g_gemm_variant.exchange(variant);
 }
 
@@ -585,6 +707,6 @@ const char* dpo_status_string(dpo_status s) {
   return "unknown status";
 }
 
-int32_t dpo_version(void) { return 100; }
+int32_t dpo_version(void) { return 200; }
 
 }  // extern "C"

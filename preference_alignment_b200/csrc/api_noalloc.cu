@@ -12,32 +12,42 @@
 //
 // The scratch lives in the file-scope array below: every device that loads the
 // library holds it until the process exits. In host code the array's name is not
-// a device address, so its address is looked up once per device with
-// cudaGetSymbolAddress (on the first call made while that device is current) and
-// then handed to the kernels like any caller-provided workspace.
+// a device address, so its address is looked up with cudaGetSymbolAddress on the
+// first call made while that device is current (and again if the device's context
+// has been destroyed and rebuilt since, which moves the array) and then handed to
+// the kernels like any caller-provided workspace.
 #include <mutex>
 
 #include "dpo.h"
+#include "internal.h"
 
 namespace {
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[DPO_NOALLOC_SCRATCH_BYTES];
 
+struct ScratchAddr {
+  void* ctx = nullptr;
+  void* ptr = nullptr;
+};
 std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[256] = {};
+ScratchAddr g_noalloc[256];
 
-// Device address of the scratch array on the current device (looked up once).
+// Device address of the scratch array on the current device, cached per context.
 dpo_status noalloc_scratch(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 256) return DPO_ERR_CUDA;
+  void* ctx = nullptr;
+  if (!dpo::current_context(&ctx)) return DPO_ERR_CUDA;
   std::lock_guard<std::mutex> lk(g_noalloc_mu);
-  if (g_noalloc_ptr[dev] == nullptr) {
+  ScratchAddr& a = g_noalloc[dev];
+  if (a.ptr == nullptr || a.ctx != ctx) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
       return DPO_ERR_CUDA;
-    g_noalloc_ptr[dev] = p;
+    a.ptr = p;
+    a.ctx = ctx;
   }
-  *out = g_noalloc_ptr[dev];
+  *out = a.ptr;
   return DPO_OK;
 }
 

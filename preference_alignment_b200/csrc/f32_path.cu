@@ -129,12 +129,13 @@ cudaError_t launch_f32_dh(const float* G, const float* W, const Sched& s, int to
   return cudaGetLastError();
 }
 
-// dW[v, k] (+)= sum_i G[i, v] H[dst[tok0 + i], k]; one block per vocab row.
+// dW[v, k] (+)= sum_i G[i, v] H[dst[tok0 + i], k] for v in [v0, v0 + gridDim.x);
+// one block per vocab row.
 __global__ void __launch_bounds__(256) k_f32_dw(const float* __restrict__ G,
                                                 const float* __restrict__ H, Sched s, int tok0,
-                                                int Mc, int d, int V, float* __restrict__ dW,
-                                                int accumulate) {
-  const int v = blockIdx.x;
+                                                int Mc, int d, int V, int v0,
+                                                float* __restrict__ dW, int accumulate) {
+  const int v = v0 + blockIdx.x;
   float* o = dW + static_cast<long long>(v) * d;
   for (int k = threadIdx.x; k < d; k += blockDim.x) {
     double a = 0.0;     // fp64: Mc products per element
@@ -146,9 +147,9 @@ __global__ void __launch_bounds__(256) k_f32_dw(const float* __restrict__ G,
 }
 
 cudaError_t launch_f32_dw(const float* G, const float* H, const Sched& s, int tok0, int Mc, int d,
-                          int V, float* dW, int accumulate, cudaStream_t st) {
-  if (V == 0) return cudaSuccess;
-  k_f32_dw<<<V, 256, 0, st>>>(G, H, s, tok0, Mc, d, V, dW, accumulate);
+                          int V, int v0, int v1, float* dW, int accumulate, cudaStream_t st) {
+  if (v1 <= v0) return cudaSuccess;
+  k_f32_dw<<<v1 - v0, 256, 0, st>>>(G, H, s, tok0, Mc, d, V, v0, dW, accumulate);
   return cudaGetLastError();
 }
 

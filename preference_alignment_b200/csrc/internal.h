@@ -54,7 +54,7 @@ struct Sched {
   int* y;                 // [Nc] target token of each scored position (-1 = out of range)
   int* dst;               // [Nc] flat index r * L + t of each scored position
   int* rowid;             // [Nc] row of each scored position
-  int* sync;              // [kSyncInts] pacing counters of the GEMM launches
+  int* sync;              // [kSyncInts] the GEMM launches' tile claim counter
 };
 
 cudaError_t launch_upload_rows(const RowChunk& rc, int* row_start, int* prompt,
@@ -105,10 +105,11 @@ cudaError_t launch_bwd_dw(const CUtensorMap& mapA, const CUtensorMap& mapB, int 
                           float* dW, int accumulate, int grid, int* sync, const DevCtl& ctl,
                           cudaStream_t st);
 
-// Loss kernel (fp64 inside).
+// Loss kernel (fp64 inside). pairs_total / nll_tokens_total: the whole data-parallel
+// batch's pair count and chosen-token count (0: this call's own).
 cudaError_t launch_loss(int B, int layout, const float* pol, const float* ref, double beta,
                         double grad_scale, int normalize, double nll_weight, const int* clen,
-                        float* loss, float* accuracy, float* margins, float* chosen_rewards,
+                        long long pairs_total, long long nll_tokens_total, float* loss, float* accuracy, float* margins, float* chosen_rewards,
                         float* rejected_rewards, float* weights, float* row_coef, float* nll,
                         cudaStream_t st);
 
@@ -120,18 +121,25 @@ cudaError_t launch_f32_grad(const float* H, const float* W, const Sched& s, int 
                             cudaStream_t st);
 cudaError_t launch_f32_dh(const float* G, const float* W, const Sched& s, int tok0, int Mc, int d,
                           int V, float* dH, cudaStream_t st);
+// dW rows [v0, v1) (dW points at the whole [V, d] array).
 cudaError_t launch_f32_dw(const float* G, const float* H, const Sched& s, int tok0, int Mc, int d,
-                          int V, float* dW, int accumulate, cudaStream_t st);
+                          int V, int v0, int v1, float* dW, int accumulate, cudaStream_t st);
 
 // 64-bit order-independent fingerprint of a device buffer into out (device).
 cudaError_t launch_fingerprint(const void* data, unsigned long long bytes,
                                unsigned long long* out, int sms, cudaStream_t st);
 
-// GEMM kernel selection, one bit per GEMM kind (dpo_set_gemm_variant): a set bit
-// runs that GEMM on the single-CTA kernel, a clear bit on CTA pairs when the device
-// can co-schedule them.
+// GEMM kernel selection (dpo_set_gemm_variant), two bits per GEMM kind: bit `kind` set
+// runs that GEMM on the single-CTA kernel (clear: CTA pairs when the device can
+// co-schedule them); bit 4 + kind set gives the pair kernel the static tile schedule
+// (clear: tiles claimed in raster order).
 enum GemmKind : int { kGemmForward = 0, kGemmGrad = 1, kGemmDH = 2, kGemmDW = 3 };
 int gemm_variant();
+
+// The CUDA context current on this thread (false if none or the driver call failed).
+// Device addresses of the library's file-scope arrays are cached per context: a
+// context that is destroyed and rebuilt reloads the module at new addresses.
+bool current_context(void** ctx);
 
 // Bounded-wait self-test: one CTA waits on an mbarrier nothing arrives on.
 cudaError_t launch_wait_selftest(const DevCtl& ctl, cudaStream_t st);

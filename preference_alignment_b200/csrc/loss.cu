@@ -8,6 +8,12 @@
 // computes", rewards/margin/weight in "A worked example of the numbers", the
 // mean and reward accuracy of dpo_step in "A training configuration that fits".)
 // row_coef[row] = d(grad_scale * loss)/d pi_row = -/+ grad_scale * beta * w / B.
+//
+// Data-parallel shares: with pairs_total = B_g (the pairs of the whole batch over
+// every rank) the batch means divide by B_g instead of this call's B, and with
+// nll_tokens_total = N_g the NLL term divides by the whole batch's chosen tokens, so
+// loss, accuracy, nll and row_coef are this rank's share of the global values: their
+// sum over ranks equals the single-process result on the whole batch.
 #include <cmath>
 
 #include "internal.h"
@@ -27,7 +33,8 @@ __device__ __forceinline__ double sigmoid_d(double x) {
 __global__ void __launch_bounds__(256) k_dpo_loss(int B, int layout, const float* __restrict__ pol,
                                                   const float* __restrict__ ref, double beta,
                                                   double gscale, int normalize, double nll_w,
-                                                  const int* __restrict__ clen, float* loss,
+                                                  const int* __restrict__ clen, double pairs_div,
+                                                  double ntok_total, float* loss,
                                                   float* accuracy, float* margins,
                                                   float* chosen_rewards, float* rejected_rewards,
                                                   float* weights, float* row_coef, float* nll_out) {
@@ -60,7 +67,7 @@ __global__ void __launch_bounds__(256) k_dpo_loss(int B, int layout, const float
     if (rejected_rewards) rejected_rewards[i] = static_cast<float>(beta * rho_r);
     if (weights) weights[i] = static_cast<float>(w);
     if (row_coef) {
-      const double k = gscale * beta * w / B;
+      const double k = gscale * beta * w / pairs_div;
       row_coef[c] = static_cast<float>(-k * sc);
       row_coef[r] = static_cast<float>(k * sr);
     }
@@ -80,11 +87,12 @@ __global__ void __launch_bounds__(256) k_dpo_loss(int B, int layout, const float
     __syncthreads();
   }
   // NLL of the chosen completions: mean over all their tokens, from the raw sums
-  const double ntok = s_den[0];
+  // (over the whole batch's chosen tokens when ntok_total > 0)
+  const double ntok = ntok_total > 0.0 ? ntok_total : s_den[0];
   const double nll = (nll_w != 0.0 && ntok > 0.0) ? -s_num[0] / ntok : 0.0;
   if (threadIdx.x == 0) {
-    *loss = static_cast<float>(s_loss[0] / B + nll_w * nll);
-    if (accuracy) *accuracy = static_cast<float>(s_acc[0] / B);
+    *loss = static_cast<float>(s_loss[0] / pairs_div + nll_w * nll);
+    if (accuracy) *accuracy = static_cast<float>(s_acc[0] / pairs_div);
     if (nll_out) *nll_out = static_cast<float>(nll);
   }
   if (row_coef && nll_w != 0.0 && ntok > 0.0) {
@@ -99,12 +107,14 @@ __global__ void __launch_bounds__(256) k_dpo_loss(int B, int layout, const float
 
 cudaError_t launch_loss(int B, int layout, const float* pol, const float* ref, double beta,
                         double grad_scale, int normalize, double nll_weight, const int* clen,
-                        float* loss, float* accuracy, float* margins, float* chosen_rewards,
+                        long long pairs_total, long long nll_tokens_total, float* loss,
+                        float* accuracy, float* margins, float* chosen_rewards,
                         float* rejected_rewards, float* weights, float* row_coef, float* nll,
                         cudaStream_t st) {
+  const double pairs_div = static_cast<double>(pairs_total > 0 ? pairs_total : B);
   k_dpo_loss<<<1, 256, 0, st>>>(B, layout, pol, ref, beta, grad_scale, normalize, nll_weight, clen,
-                                loss, accuracy, margins, chosen_rewards, rejected_rewards, weights,
-                                row_coef, nll);
+                                pairs_div, static_cast<double>(nll_tokens_total), loss, accuracy,
+                                margins, chosen_rewards, rejected_rewards, weights, row_coef, nll);
   return cudaGetLastError();
 }
 

@@ -1,25 +1,92 @@
 """Data-parallel exchange of the DPO head step.
 
 Each rank scores its own pairs (both rows of a pair stay on one rank) with the
-same weights. The loss is the mean over all pairs of all ranks, so each rank
-folds 1/world_size into the per-row coefficients (dpo_loss's grad_scale), and
-the step's one exchange is a sum all-reduce of dW (and of the loss, then divided
-by world_size). dH stays on its rank. This mirrors the data-parallel replicas of
-the pages' systems ("Run Distributed Full-Model DPO with PyTorch FSDP", Step 1;
-Megatron-Bridge PR 6092, the DP replicas of its results), at the LM head.
+same weights; ranks may hold different numbers of pairs and tokens. The loss is
+the mean over all pairs of all ranks (and the NLL term, when used, the mean over
+all chosen completion tokens of all ranks), so:
+
+1. `global_counts` sums the pair and chosen-token counts over the ranks;
+2. every rank calls dpo_loss_ex with those totals (pairs_total, nll_tokens_total):
+   its loss, accuracy, NLL and row coefficients are then its share of the whole
+   batch's values, exact for unequal shards;
+3. the backward's one exchange is a sum all-reduce of dW. `backward_exchange`
+   forms dW block by block of vocabulary rows (dpo_backward_dw) and starts the
+   all-reduce of each finished block while the next one is computed, then forms
+   dH, which needs no exchange, while the last block's all-reduce runs;
+4. `allreduce_shares` sums the loss shares (one small all-reduce).
+
+dH stays on its rank. This mirrors the data-parallel replicas of the pages'
+systems ("Run Distributed Full-Model DPO with PyTorch FSDP", Step 1: every rank
+holds part of the global batch and the gradients are summed; Megatron-Bridge PR
+6092, the DP replicas of its results), at the LM head.
 """
 from __future__ import annotations
 
+# Vocabulary rows per dW block are whole 256-row tiles of the dW GEMM (its M tiles),
+# so a block boundary never splits a tile.
+ROW_ALIGN = 256
 
-def grad_scale(world_size: int, accumulation_steps: int = 1) -> float:
-    """grad_scale for dpo_loss so that summed per-rank gradients are those of the global mean."""
-    return 1.0 / (world_size * accumulation_steps)
 
-
-def allreduce_step(dW, loss, group=None):
-    """Sum dW over ranks in place; turn the per-rank mean losses into the global mean."""
+def global_counts(pairs: int, chosen_tokens: int, group=None, device=None):
+    """(pairs, chosen completion tokens) summed over the ranks of `group`."""
+    import torch
     import torch.distributed as dist
-    ws = dist.get_world_size(group)
-    dist.all_reduce(dW, group=group)
-    dist.all_reduce(loss, group=group)
-    loss.mul_(1.0 / ws)
+    t = torch.tensor([int(pairs), int(chosen_tokens)], dtype=torch.int64, device=device)
+    dist.all_reduce(t, group=group)
+    return int(t[0]), int(t[1])
+
+
+def vocab_buckets(V: int, n_buckets: int, align: int = ROW_ALIGN):
+    """Split vocabulary rows [0, V) into at most n_buckets contiguous blocks whose
+    boundaries are multiples of `align` (the last block ends at V)."""
+    if V < 1 or n_buckets < 1:
+        raise ValueError("V and n_buckets must be positive")
+    tiles = (V + align - 1) // align
+    n = min(n_buckets, tiles)
+    edges = [min(V, (tiles * b // n) * align) for b in range(n + 1)]
+    return [(edges[b], edges[b + 1]) for b in range(n) if edges[b + 1] > edges[b]]
+
+
+def bucketed_allreduce(dW, buckets, compute_bucket, group=None):
+    """For each block (v0, v1): compute_bucket(v0, v1) fills dW[v0:v1] on the current
+    stream, then an asynchronous sum all-reduce of those rows starts (on NCCL it
+    waits only for the work already enqueued, so it runs while the next block is
+    computed). Returns the pending works; call finish(works) before using dW."""
+    import torch.distributed as dist
+    works = []
+    for v0, v1 in buckets:
+        compute_bucket(v0, v1)
+        works.append(dist.all_reduce(dW[v0:v1], group=group, async_op=True))
+    return works
+
+
+def finish(works):
+    """Make the current stream (NCCL) or the host (gloo) wait for the pending all-reduces."""
+    for w in works:
+        w.wait()
+
+
+def allreduce_shares(shares, group=None):
+    """Sum per-rank shares (e.g. [loss, accuracy, nll]) in place: the whole batch's values."""
+    import torch.distributed as dist
+    dist.all_reduce(shares, group=group)
+    return shares
+
+
+def backward_exchange(batch, lse_state, row_coef, dH, dW, ws, n_buckets=8, max_sms=0,
+                      group=None):
+    """The data-parallel backward on this rank: dz once (dpo_backward with dW = NULL),
+    then dW block by block with each block's all-reduce started as soon as it is
+    formed, then dH while the last all-reduce runs. max_sms > 0 leaves the other SMs
+    free for the collective's kernels. Everything is enqueued on torch's current
+    stream, the stream the collectives order against. Returns the pending works
+    (finish() them)."""
+    from preference_alignment_b200 import libdpo
+    libdpo.backward(batch, lse_state, row_coef, None, None, False, ws)
+    works = bucketed_allreduce(
+        dW, vocab_buckets(int(batch.c.V), n_buckets),
+        lambda v0, v1: libdpo.backward_dw(batch, v0, v1, dW, False, ws, max_sms=max_sms),
+        group=group)
+    if dH is not None:
+        libdpo.backward_dh(batch, dH, ws, max_sms=max_sms)
+    return works

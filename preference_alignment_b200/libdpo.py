@@ -178,20 +178,25 @@ def loss(B: int, layout, pol, ref, beta: float, grad_scale: float, loss_out, acc
 
 class LossOptions(ctypes.Structure):
     _fields_ = [("normalize", ctypes.c_int32), ("nll_weight", ctypes.c_float),
-                ("completion_len", ctypes.c_void_p)]
+                ("completion_len", ctypes.c_void_p), ("pairs_total", ctypes.c_int32),
+                ("nll_tokens_total", ctypes.c_int64)]
 
 
 def loss_ex(B: int, layout, pol, ref, beta: float, grad_scale: float, loss_out, accuracy=None,
             margins=None, chosen_rewards=None, rejected_rewards=None, weights=None, row_coef=None,
-            nll=None, normalize=False, nll_weight=0.0, completion_len=None, stream=None):
-    """dpo_loss_ex: length-normalised and/or SFT-NLL variants (completion_len: device int32 [2B])."""
+            nll=None, normalize=False, nll_weight=0.0, completion_len=None, pairs_total=0,
+            nll_tokens_total=0, stream=None):
+    """dpo_loss_ex: length-normalised and/or SFT-NLL variants (completion_len: device int32 [2B]);
+    pairs_total / nll_tokens_total > 0 make the outputs this rank's share of a data-parallel
+    batch of that many pairs / chosen tokens."""
     lib = load()
     fn = lib.dpo_loss_ex
     vp = ctypes.c_void_p
     fn.argtypes = [ctypes.c_int32, ctypes.c_int32, vp, vp, ctypes.c_float, ctypes.c_float,
                    ctypes.POINTER(LossOptions), vp, vp, vp, vp, vp, vp, vp, vp, vp]
     fn.restype = ctypes.c_int
-    opt = LossOptions(1 if normalize else 0, float(nll_weight), _ptr(completion_len))
+    opt = LossOptions(1 if normalize else 0, float(nll_weight), _ptr(completion_len),
+                      int(pairs_total), int(nll_tokens_total))
     lay = LAYOUTS[layout] if isinstance(layout, str) else int(layout)
     _check(fn(int(B), lay, _ptr(pol), _ptr(ref), float(beta), float(grad_scale), ctypes.byref(opt),
               _ptr(loss_out), _ptr(accuracy), _ptr(margins), _ptr(chosen_rewards),
@@ -204,6 +209,32 @@ def backward(batch: BatchArgs, lse_state, row_coef, dH, dW, accumulate_dW: bool,
     _check(load().dpo_backward(ctypes.byref(batch.c), _ptr(lse_state), _ptr(row_coef), _ptr(dH),
                                _ptr(dW), 1 if accumulate_dW else 0, _ptr(ws),
                                _nbytes(ws, ws_bytes), _stream(stream)), "dpo_backward")
+
+
+def backward_dw(batch: BatchArgs, v_begin: int, v_end: int, dW, accumulate_dW: bool, ws,
+                ws_bytes=None, max_sms: int = 0, stream=None):
+    """dpo_backward_dw: rows [v_begin, v_end) of dW from the dz a preceding
+    backward(dW=None) left in the workspace ws (max_sms > 0 caps the SMs it uses)."""
+    lib = load()
+    fn = lib.dpo_backward_dw
+    vp = ctypes.c_void_p
+    fn.argtypes = [ctypes.POINTER(Batch), ctypes.c_int32, ctypes.c_int32, vp, ctypes.c_int,
+                   ctypes.c_int32, vp, ctypes.c_size_t, vp]
+    fn.restype = ctypes.c_int
+    _check(fn(ctypes.byref(batch.c), int(v_begin), int(v_end), _ptr(dW),
+              1 if accumulate_dW else 0, int(max_sms), _ptr(ws), _nbytes(ws, ws_bytes),
+              _stream(stream)), "dpo_backward_dw")
+
+
+def backward_dh(batch: BatchArgs, dH, ws, ws_bytes=None, max_sms: int = 0, stream=None):
+    """dpo_backward_dh: dH (fully written) from the dz a preceding backward(dW=None) left in ws."""
+    lib = load()
+    fn = lib.dpo_backward_dh
+    vp = ctypes.c_void_p
+    fn.argtypes = [ctypes.POINTER(Batch), vp, ctypes.c_int32, vp, ctypes.c_size_t, vp]
+    fn.restype = ctypes.c_int
+    _check(fn(ctypes.byref(batch.c), _ptr(dH), int(max_sms), _ptr(ws), _nbytes(ws, ws_bytes),
+              _stream(stream)), "dpo_backward_dh")
 
 
 class VocabShard(ctypes.Structure):
@@ -284,7 +315,8 @@ def fingerprint(data, nbytes, out, stream=None):
 
 
 def set_gemm_variant(variant: int) -> int:
-    """Mask, one bit per GEMM (forward, dz, dH, dW): a set bit runs it on the single-CTA kernel."""
+    """Mask per GEMM k (forward, dz, dH, dW): bit k runs it on the single-CTA kernel, bit 4 + k
+    gives the CTA-pair kernel the static tile schedule instead of tiles claimed in raster order."""
     lib = load()
     fn = lib.dpo_set_gemm_variant
     fn.argtypes = [ctypes.c_int32]

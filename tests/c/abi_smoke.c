@@ -4,6 +4,11 @@
  *   abi_smoke gpu    one DPO step on the current GPU with policy == reference:
  *                    the loss must be ln 2, every weight 1/2, the accuracy 0,
  *                    and no device error may be reported.
+ *   abi_smoke case DIR   one DPO step (policy forward, reference forward, loss,
+ *                    backward) on the inputs in DIR, checked against the expected
+ *                    values in DIR (written by the Python test from the fp64 oracle):
+ *                    sequence sums |err| <= 5e-2 and <= 1e-4 relative, loss |err|
+ *                    <= 1e-4, dH and dW relative Frobenius error <= 1e-2.
  * Exit status 0 on success; the failing check is printed otherwise. */
 #include <math.h>
 #include <stdio.h>
@@ -114,7 +119,122 @@ static int gpu_step(void) {
   return 0;
 }
 
+/* Read exactly n bytes of DIR/name into a new host buffer (NULL on failure). */
+static void* read_file(const char* dir, const char* name, size_t n) {
+  char path[4096];
+  snprintf(path, sizeof path, "%s/%s", dir, name);
+  FILE* f = fopen(path, "rb");
+  if (!f) return NULL;
+  void* p = malloc(n > 0 ? n : 1);
+  size_t got = fread(p, 1, n, f);
+  fclose(f);
+  if (got != n) {
+    free(p);
+    return NULL;
+  }
+  return p;
+}
+
+/* Relative Frobenius error of a float array against a double array. */
+static double rel_frob(const float* a, const double* b, size_t n) {
+  double num = 0.0, den = 0.0;
+  for (size_t i = 0; i < n; ++i) {
+    const double e = (double)a[i] - b[i];
+    num += e * e;
+    den += b[i] * b[i];
+  }
+  return sqrt(num / (den > 0.0 ? den : 1e-300));
+}
+
+static int case_step(const char* dir) {
+  /* meta: R L d V beta (pairs in halves layout) */
+  char path[4096];
+  snprintf(path, sizeof path, "%s/meta.txt", dir);
+  FILE* mf = fopen(path, "r");
+  CHECK(mf != NULL);
+  int R = 0, L = 0, d = 0, V = 0;
+  double beta = 0.0;
+  CHECK(fscanf(mf, "%d %d %d %d %lf", &R, &L, &d, &V, &beta) == 5);
+  fclose(mf);
+  CHECK(R > 0 && R % 2 == 0 && L > 1 && d > 0 && V > 0);
+  const int B = R / 2;
+  const size_t nh = (size_t)R * L * d, nw = (size_t)V * d;
+  uint16_t* h = (uint16_t*)read_file(dir, "H.bin", nh * 2);
+  uint16_t* w = (uint16_t*)read_file(dir, "W.bin", nw * 2);
+  uint16_t* wr = (uint16_t*)read_file(dir, "W_ref.bin", nw * 2);
+  int32_t* tok = (int32_t*)read_file(dir, "tokens.bin", sizeof(int32_t) * R * L);
+  int32_t* P = (int32_t*)read_file(dir, "prompt_len.bin", sizeof(int32_t) * R);
+  int32_t* C = (int32_t*)read_file(dir, "completion_len.bin", sizeof(int32_t) * R);
+  double* e_pol = (double*)read_file(dir, "pol.bin", sizeof(double) * R);
+  double* e_ref = (double*)read_file(dir, "ref.bin", sizeof(double) * R);
+  double* e_loss = (double*)read_file(dir, "loss.bin", sizeof(double));
+  double* e_dH = (double*)read_file(dir, "dH.bin", sizeof(double) * nh);
+  double* e_dW = (double*)read_file(dir, "dW.bin", sizeof(double) * nw);
+  CHECK(h && w && wr && tok && P && C && e_pol && e_ref && e_loss && e_dH && e_dW);
+
+  void *dHin, *dWin, *dWr, *dtok, *ws, *dlse, *dpol, *dref, *dloss, *dcoef, *ddH, *ddW;
+  CHECK(cudaMalloc(&dHin, nh * 2) == cudaSuccess);
+  CHECK(cudaMalloc(&dWin, nw * 2) == cudaSuccess);
+  CHECK(cudaMalloc(&dWr, nw * 2) == cudaSuccess);
+  CHECK(cudaMalloc(&dtok, sizeof(int32_t) * R * L) == cudaSuccess);
+  CHECK(cudaMemcpy(dHin, h, nh * 2, cudaMemcpyHostToDevice) == cudaSuccess);
+  CHECK(cudaMemcpy(dWin, w, nw * 2, cudaMemcpyHostToDevice) == cudaSuccess);
+  CHECK(cudaMemcpy(dWr, wr, nw * 2, cudaMemcpyHostToDevice) == cudaSuccess);
+  CHECK(cudaMemcpy(dtok, tok, sizeof(int32_t) * R * L, cudaMemcpyHostToDevice) == cudaSuccess);
+
+  dpo_batch b, br;
+  memset(&b, 0, sizeof b);
+  b.R = R; b.L = L; b.d = d; b.V = V; b.dtype = DPO_BF16;
+  b.H = dHin; b.W = dWin; b.tokens = (const int32_t*)dtok;
+  b.prompt_len = P; b.completion_len = C;
+  br = b;
+  br.W = dWr;
+  size_t f = 0, bw = 0;
+  CHECK(dpo_workspace_size(&b, &f, &bw, NULL) == DPO_OK);
+  const size_t wsb = f > bw ? f : bw;
+  int nc = 0;
+  for (int r = 0; r < R; ++r) nc += C[r];
+  CHECK(cudaMalloc(&ws, wsb) == cudaSuccess);
+  CHECK(cudaMalloc(&dlse, sizeof(float) * (nc > 0 ? nc : 1)) == cudaSuccess);
+  CHECK(cudaMalloc(&dpol, sizeof(float) * R) == cudaSuccess);
+  CHECK(cudaMalloc(&dref, sizeof(float) * R) == cudaSuccess);
+  CHECK(cudaMalloc(&dloss, sizeof(float)) == cudaSuccess);
+  CHECK(cudaMalloc(&dcoef, sizeof(float) * R) == cudaSuccess);
+  CHECK(cudaMalloc(&ddH, sizeof(float) * nh) == cudaSuccess);
+  CHECK(cudaMalloc(&ddW, sizeof(float) * nw) == cudaSuccess);
+
+  CHECK(dpo_seq_logprobs(&b, 1, (float*)dpol, NULL, (float*)dlse, ws, wsb, NULL) == DPO_OK);
+  CHECK(dpo_seq_logprobs(&br, 0, (float*)dref, NULL, NULL, ws, wsb, NULL) == DPO_OK);
+  CHECK(dpo_loss(B, DPO_PAIRS_HALVES, (float*)dpol, (float*)dref, (float)beta, 1.0f,
+                 (float*)dloss, NULL, NULL, NULL, NULL, NULL, (float*)dcoef, NULL) == DPO_OK);
+  CHECK(dpo_backward(&b, (float*)dlse, (float*)dcoef, (float*)ddH, (float*)ddW, 0, ws, wsb,
+                     NULL) == DPO_OK);
+  CHECK(dpo_check(NULL) == DPO_OK);
+
+  float* pol = (float*)malloc(sizeof(float) * R);
+  float* ref = (float*)malloc(sizeof(float) * R);
+  float* gH = (float*)malloc(sizeof(float) * nh);
+  float* gW = (float*)malloc(sizeof(float) * nw);
+  float loss = 0.f;
+  CHECK(cudaMemcpy(pol, dpol, sizeof(float) * R, cudaMemcpyDeviceToHost) == cudaSuccess);
+  CHECK(cudaMemcpy(ref, dref, sizeof(float) * R, cudaMemcpyDeviceToHost) == cudaSuccess);
+  CHECK(cudaMemcpy(&loss, dloss, sizeof(float), cudaMemcpyDeviceToHost) == cudaSuccess);
+  CHECK(cudaMemcpy(gH, ddH, sizeof(float) * nh, cudaMemcpyDeviceToHost) == cudaSuccess);
+  CHECK(cudaMemcpy(gW, ddW, sizeof(float) * nw, cudaMemcpyDeviceToHost) == cudaSuccess);
+  for (int r = 0; r < R; ++r) {
+    const double ep = fabs((double)pol[r] - e_pol[r]), er = fabs((double)ref[r] - e_ref[r]);
+    CHECK(ep <= 5e-2 && ep <= 1e-4 * fmax(1.0, fabs(e_pol[r])));
+    CHECK(er <= 5e-2 && er <= 1e-4 * fmax(1.0, fabs(e_ref[r])));
+  }
+  CHECK(fabs((double)loss - e_loss[0]) <= 1e-4);
+  const double rh = rel_frob(gH, e_dH, nh), rw = rel_frob(gW, e_dW, nw);
+  CHECK(rh <= 1e-2 && rw <= 1e-2);
+  printf("case ok: loss %.7f (oracle %.7f), dH rel %.2e, dW rel %.2e\n", loss, e_loss[0], rh, rw);
+  return 0;
+}
+
 int main(int argc, char** argv) {
   if (argc > 1 && strcmp(argv[1], "gpu") == 0) return gpu_step();
+  if (argc > 2 && strcmp(argv[1], "case") == 0) return case_step(argv[2]);
   return host_checks();
 }

@@ -46,7 +46,7 @@ def test_status_strings_and_version(lib):
     for code in range(7):
         assert libdpo.status_string(code)
     assert libdpo.status_string(99) == "unknown status"
-    assert libdpo.version() == 100
+    assert libdpo.version() == 200
 
 
 FAKE = 0x10000  # never dereferenced: every call below fails its host checks first
@@ -109,9 +109,15 @@ def test_calls_fail_on_the_host_and_leave_outputs_alone(lib):
     with pytest.raises(libdpo.DpoError) as e:   # want_grad without lse_state
         libdpo.seq_logprobs(b, True, out, None, None, FAKE, ws_bytes=1 << 30)
     assert e.value.status == libdpo.ERR_INVALID_ARG
-    with pytest.raises(libdpo.DpoError) as e:   # backward without dW
-        libdpo.backward(b, FAKE, FAKE, None, None, False, FAKE, ws_bytes=1 << 30)
+    with pytest.raises(libdpo.DpoError) as e:   # backward without row coefficients
+        libdpo.backward(b, FAKE, None, None, FAKE, False, FAKE, ws_bytes=1 << 30)
     assert e.value.status == libdpo.ERR_INVALID_ARG
+    bl = _batch(L=128, C=[100, 100, 100, 100])    # 400 scored positions: chunked below bwd
+    _, bwl, mnl = libdpo.workspace_size(bl)
+    assert mnl < bwl
+    with pytest.raises(libdpo.DpoError) as e:   # dW deferred, but dz would not stay whole
+        libdpo.backward(bl, FAKE, FAKE, None, None, False, FAKE, ws_bytes=mnl)
+    assert e.value.status == libdpo.ERR_WORKSPACE
     f, bw, mn = libdpo.workspace_size(b)
     with pytest.raises(libdpo.DpoError) as e:   # backward workspace below the minimum
         libdpo.backward(b, FAKE, FAKE, None, FAKE, False, FAKE, ws_bytes=mn - 256)
@@ -129,6 +135,44 @@ def test_loss_rejects(lib, args):
     with pytest.raises(libdpo.DpoError) as e:
         libdpo.loss(a["B"], a["layout"], a["pol"], a["ref"], a["beta"], a["grad_scale"],
                     a["loss_out"])
+    assert e.value.status == libdpo.ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("v0,v1,dW,max_sms,ws,code", [
+    (4, 96, FAKE, 0, 1 << 30, libdpo.ERR_INVALID_ARG),     # v_begin not a multiple of 8
+    (0, 101, FAKE, 0, 1 << 30, libdpo.ERR_INVALID_ARG),    # past V
+    (16, 8, FAKE, 0, 1 << 30, libdpo.ERR_INVALID_ARG),     # empty-reversed range
+    (0, 90, FAKE, 0, 1 << 30, libdpo.ERR_INVALID_ARG),     # v_end neither 8k nor V
+    (0, 100, None, 0, 1 << 30, libdpo.ERR_INVALID_ARG),    # no dW
+    (0, 100, FAKE, -1, 1 << 30, libdpo.ERR_INVALID_ARG),   # negative SM budget
+    (0, 100, FAKE, 0, 0, libdpo.ERR_WORKSPACE),            # no workspace
+])
+def test_backward_dw_rejects(lib, v0, v1, dW, max_sms, ws, code):
+    b = _batch()
+    with pytest.raises(libdpo.DpoError) as e:
+        libdpo.backward_dw(b, v0, v1, dW, False, FAKE if ws else 0, ws_bytes=ws, max_sms=max_sms)
+    assert e.value.status == code
+
+
+def test_backward_dh_and_dw_need_the_whole_dz(lib):
+    b = _batch(L=128, C=[100, 100, 100, 100])
+    _, bw, mn = libdpo.workspace_size(b)
+    with pytest.raises(libdpo.DpoError) as e:
+        libdpo.backward_dw(b, 0, 100, FAKE, False, FAKE, ws_bytes=mn)
+    assert e.value.status == libdpo.ERR_WORKSPACE
+    with pytest.raises(libdpo.DpoError) as e:
+        libdpo.backward_dh(b, FAKE, FAKE, ws_bytes=bw - 256)
+    assert e.value.status == libdpo.ERR_WORKSPACE
+    with pytest.raises(libdpo.DpoError) as e:
+        libdpo.backward_dh(b, None, FAKE, ws_bytes=bw)
+    assert e.value.status == libdpo.ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("kw", [dict(pairs_total=1), dict(pairs_total=-3),
+                                dict(nll_tokens_total=-1)])
+def test_loss_ex_rejects_bad_data_parallel_counts(lib, kw):
+    with pytest.raises(libdpo.DpoError) as e:
+        libdpo.loss_ex(2, "halves", FAKE, FAKE, 0.1, 1.0, FAKE, **kw)
     assert e.value.status == libdpo.ERR_INVALID_ARG
 
 

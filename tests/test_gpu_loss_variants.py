@@ -12,7 +12,8 @@ from dpo_harness import DeviceWorkload, TOL_GRAD, TOL_LOSS, np64, rel_frob
 pytestmark = pytest.mark.gpu
 
 
-def _run_ex(B, layout, pol, ref, C, beta, gscale, normalize, nll_weight):
+def _run_ex(B, layout, pol, ref, C, beta, gscale, normalize, nll_weight, pairs_total=0,
+            nll_tokens_total=0):
     import torch
     dev = "cuda"
     t = lambda a: torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(dev)  # noqa: E731
@@ -22,7 +23,8 @@ def _run_ex(B, layout, pol, ref, C, beta, gscale, normalize, nll_weight):
     clen = torch.from_numpy(np.asarray(C, np.int32)).to(dev)
     libdpo.loss_ex(B, layout, t(pol), t(ref), beta, gscale, out["loss"], out["acc"], out["m"],
                    out["cr"], out["rr"], out["w"], out["coef"], out["nll"], normalize=normalize,
-                   nll_weight=nll_weight, completion_len=clen)
+                   nll_weight=nll_weight, completion_len=clen, pairs_total=pairs_total,
+                   nll_tokens_total=nll_tokens_total)
     return {k: np64(v) for k, v in out.items()}
 
 
@@ -70,3 +72,34 @@ def test_variants_end_to_end_through_the_backward():
     oH, oW = O.backward(H, Wd, w.tokens, w.prompt_len, w.completion_len, ol["row_coef"])
     assert rel_frob(np64(dH), oH) <= TOL_GRAD
     assert rel_frob(np64(dW), oW) <= TOL_GRAD
+
+
+@pytest.mark.parametrize("normalize,nll", [(False, 0.0), (False, 0.5), (True, 0.25)])
+def test_data_parallel_shares_against_the_oracle(normalize, nll):
+    """dpo_loss_ex with the whole batch's pair and chosen-token counts: each part of an
+    unequal partition gives the oracle's share, and the shares add up to the oracle's
+    single-process values of the whole batch."""
+    rng = np.random.default_rng(73)
+    B = 9
+    C = rng.integers(1, 500, 2 * B)
+    pol = (-rng.uniform(0.5, 4.0, 2 * B) * C).astype(np.float32)
+    ref = (pol + rng.normal(0, 5, 2 * B)).astype(np.float32)
+    Ng = int(C[0::2].sum())
+    whole = O.dpo_loss(pol.astype(np.float64), ref.astype(np.float64), 0.1, "adjacent",
+                       completion_len=C, normalize=normalize, nll_weight=nll)
+    tot = np.zeros(3)
+    for pairs in ([0, 1, 2, 3, 4, 5], [6], [7, 8]):
+        rows = np.array([r for i in pairs for r in (2 * i, 2 * i + 1)])
+        o = O.dpo_loss(pol[rows].astype(np.float64), ref[rows].astype(np.float64), 0.1,
+                       "adjacent", completion_len=C[rows], normalize=normalize, nll_weight=nll,
+                       pairs_total=B, nll_tokens_total=Ng)
+        g = _run_ex(len(pairs), "adjacent", pol[rows], ref[rows], C[rows], 0.1, 1.0, normalize,
+                    nll, pairs_total=B, nll_tokens_total=Ng)
+        assert abs(g["loss"][0] - o["loss"]) <= TOL_LOSS
+        assert g["acc"][0] == pytest.approx(o["accuracy"], abs=1e-7)
+        np.testing.assert_allclose(g["coef"], o["row_coef"], rtol=1e-5, atol=1e-10)
+        np.testing.assert_allclose(g["coef"], whole["row_coef"][rows], rtol=1e-5, atol=1e-10)
+        tot += [g["loss"][0], g["acc"][0], g["nll"][0]]
+    assert abs(tot[0] - whole["loss"]) <= TOL_LOSS
+    assert tot[1] == pytest.approx(whole["accuracy"], abs=1e-6)
+    assert abs(tot[2] - whole["nll"]) <= 1e-5 * max(1.0, abs(whole["nll"]))

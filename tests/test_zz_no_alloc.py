@@ -2,14 +2,16 @@
 
 It serves callers that may not allocate device memory (a framework that owns
 the device-memory budget and forbids allocation from its plugins, or code that
-cannot accept the synchronisation cudaMalloc/cudaFree may cause). Its results
-must match dpo_seq_logprobs, which takes a caller workspace, within the tests'
-tolerances, call after call: the built-in scratch is shared and keeps the
-previous call's contents. This file is collected last on purpose.
+cannot accept the synchronisation cudaMalloc/cudaFree may cause). The forward is
+deterministic, so its results must equal those of dpo_seq_logprobs, which takes a
+caller workspace, bit for bit, call after call (the built-in scratch is shared and
+keeps the previous call's contents), and match the oracle within the path's
+tolerances. This file is collected last on purpose.
 """
 import numpy as np
 import pytest
 
+from oracle import dpo_oracle as O
 from preference_alignment_b200 import libdpo
 from preference_alignment_b200 import workloads as WL
 
@@ -36,7 +38,8 @@ def test_noalloc_matches_workspace_entry_point_on_consecutive_calls():
         WL.make_custom(R=4, L=500, d=512, V=3000, dtype="bf16", seed=32, prompt_range=(1, 100),
                        full_rows=2),
     ]
-    for w in cases:
+    import torch
+    for k, w in enumerate(cases):
         dw = DeviceWorkload(w)
         fwd, _, _ = libdpo.workspace_size(dw.batch())
         assert fwd <= libdpo.NOALLOC_SCRATCH_BYTES
@@ -44,9 +47,15 @@ def test_noalloc_matches_workspace_entry_point_on_consecutive_calls():
         seq_b, tok_b, lse_b = _noalloc(dw)                          # built-in scratch
         assert libdpo.check() == libdpo.OK
         nc = w.n_scored
-        assert np.abs(np64(tok_b) - np64(tok_a)).max() <= TOL_TOK
-        assert_seq_close(np64(seq_b), np64(seq_a))
-        assert np.abs(np64(lse_b)[:nc] - np64(lse_a)[:nc]).max() <= TOL_TOK
+        assert torch.equal(seq_b, seq_a)
+        assert torch.equal(tok_b, tok_a)
+        assert torch.equal(lse_b[:nc], lse_a[:nc])
+        if k == 0:
+            o = O.seq_logprobs(WL.widen(w.H, w.dtype), WL.widen(w.W, w.dtype), w.tokens,
+                               w.prompt_len, w.completion_len)
+            assert np.abs(np64(tok_b) - o["tok_logp"]).max() <= TOL_TOK
+            assert_seq_close(np64(seq_b), o["seq_logp"])
+            assert np.abs(np64(lse_b)[:nc] - o["lse"]).max() <= TOL_TOK
 
 
 def test_noalloc_refuses_batches_beyond_its_scratch():
