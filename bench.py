@@ -104,6 +104,19 @@ def rank_workload(name, rank, weights=True):
     return w
 
 
+def keep_pairs(w, pairs):
+    """The workload cut to its first `pairs` pairs (both rows of each), same weights."""
+    B = w.R // 2
+    if w.layout == "halves":
+        rows = np.r_[0:pairs, B:B + pairs]
+    else:
+        rows = np.arange(2 * pairs)
+    w.R = 2 * pairs
+    for k in ("prompt_len", "completion_len", "tokens", "H"):
+        setattr(w, k, np.ascontiguousarray(getattr(w, k)[rows]))
+    return w
+
+
 class ClockSampler:
     """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
 
@@ -333,12 +346,16 @@ def run_ours(args):
     libdpo.set_gemm_variant(args.gemm_variant)
 
     w = rank_workload(args.workload, rank, weights=(ws_n == 1 or rank == 0))
+    if args.pairs and args.pairs < w.R // 2:
+        w = keep_pairs(w, args.pairs)
     B = w.R // 2
 
     def dev_bf16(a):
         return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
 
-    fwd_only = not WL.CONFIGS[args.workload][9]   # offline reference scoring: forward only
+    # offline reference scoring is forward only; a profiler's forward-only run of another
+    # workload allocates only what the policy forward needs
+    fwd_only = not WL.CONFIGS[args.workload][9] or (args.profile_step > 0 and args.forward_only)
     H = dev_bf16(w.H)
     if ws_n > 1:
         # rank 0 drew the weights; the other ranks receive them (same model on every rank)
@@ -429,6 +446,15 @@ def run_ours(args):
     else:
         bwd_launches = uploads + 3 + dh_launches
     launches_per_step = (fwd_launches if fwd_only else 2 * fwd_launches + 1 + bwd_launches)
+
+    if args.profile_step:
+        # a profiler's run: the given number of plain steps, nothing timed or printed
+        for _ in range(args.profile_step):
+            step()
+        st = libdpo.check(sp)
+        if ws_n > 1:
+            dist.destroy_process_group()
+        return 0 if st == libdpo.OK else 1
 
     for _ in range(args.warmup):
         step()
@@ -658,9 +684,9 @@ def main(argv=None):
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(WL.CONFIGS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-cublas-reference", action="store_true")
-    ap.add_argument("--gemm-variant", type=int, default=0, choices=range(256),
+    ap.add_argument("--gemm-variant", type=int, default=0, choices=range(512),
                     help="mask, per GEMM (forward, dz, dH, dW) bit k: single-CTA kernel, "
-                         "bit 4 + k: static tile schedule")
+                         "bit 4 + k: static tile schedule; bit 8: dH without split-K")
     ap.add_argument("--cpu-tokens-per-row", type=int, default=64,
                     help="oracle sample (CPU baseline and reference arm): completion tokens "
                          "per row of one pair")
@@ -670,6 +696,14 @@ def main(argv=None):
                     help="data parallel: blocks of dW rows whose all-reduce overlaps the next")
     ap.add_argument("--comm-sms", type=int, default=16,
                     help="data parallel: SMs the backward GEMMs leave free for NCCL")
+    ap.add_argument("--pairs", type=int, default=0,
+                    help="keep only the workload's first P pairs (a smaller case, e.g. for a "
+                         "profiler); 0 = all")
+    ap.add_argument("--profile-step", type=int, default=0,
+                    help="run this many untimed steps and exit (a profiler's command)")
+    ap.add_argument("--forward-only", action="store_true",
+                    help="with --profile-step: the policy forward alone (weights, H and the "
+                         "forward workspace on the device, nothing else)")
     raw = sys.argv[1:] if argv is None else list(argv)
     args = ap.parse_args(raw)
     if args.warmup < 3 and args.impl == "ours":

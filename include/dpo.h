@@ -174,9 +174,11 @@ dpo_status dpo_loss_ex(int32_t B, int32_t layout, const float* pol, const float*
 /* Backward of sum_r row_coef[r] * seq_logp[r] (step 5) to H and W.
  *   lse_state   device [Nc] fp32 from dpo_seq_logprobs(want_grad=1) on the same batch
  *   row_coef    device [R] fp32, d(objective)/d seq_logp[r] (dpo_loss writes it)
- *   dH          device [R, L, d] fp32, out: fully written; 0 at unscored positions
- *   dW          device [V, d] fp32, out: dW = sum_t dz_t^T h_t, or dW += that when
- *               accumulate_dW != 0 (gradient accumulation over micro-batches)
+ *   dH          device [R, L, d] fp32, 16-byte aligned, out: fully written; 0 at
+ *               unscored positions
+ *   dW          device [V, d] fp32, 16-byte aligned, out: dW = sum_t dz_t^T h_t, or
+ *               dW += that when accumulate_dW != 0 (gradient accumulation over
+ *               micro-batches)
  *   ws          device workspace, >= bwd_min_bytes, 256-byte aligned
  * with dz[t, v] = row_coef[r(t)] * (1[v = tokens[r, t+1]] - softmax(z_t)[v]). The
  * logits are recomputed tile by tile. dH may be NULL (only dW is formed).
@@ -349,9 +351,12 @@ dpo_status dpo_selftest_wait_timeout(uint32_t budget_ms, void* stream);
  *   bit 4 + k  clear: the CTA pairs claim tiles in raster order from a counter in the
  *              workspace (the tiles in flight stay one contiguous window of the
  *              raster); set: static round-robin (pair p takes tiles p, p + pairs, ...).
- * Every choice gives the same results (each tile is computed the same way). Default
- * 0. Returns the previous mask, or -1 for a value outside 0..255. A diagnostic for
- * measurements; the default is the fastest measured. */
+ *   bit 8      set: dH = dz.W is never split over the vocabulary (K) into parts of one
+ *              launch (clear: split when that fills the GPU's waves better); this bit
+ *              also changes the backward workspace size, so set it before sizing.
+ * Every choice gives the same results within rounding (bits 4-7 bit for bit: each tile
+ * is computed the same way). Default 0. Returns the previous mask, or -1 for a value
+ * outside 0..511. A diagnostic for measurements; the default is the fastest measured. */
 int32_t dpo_set_gemm_variant(int32_t variant);
 
 /* Static description of a status code. */

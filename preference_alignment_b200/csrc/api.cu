@@ -123,10 +123,65 @@ struct Plan {
   // forward suffix
   int S = 0, ldp = 0;
   size_t off_part = 0, off_zy = 0, off_lp = 0, fwd_total = 0;
-  // backward suffix
-  size_t off_G = 0, g_row_bytes = 0, bwd_total = 0, bwd_min = 0;
+  // backward suffix: per position one dz row (g_row_bytes) and, with split-K dH, the
+  // fp32 partial sums of K parts 1.. (part_row_bytes)
+  size_t off_G = 0, g_row_bytes = 0, part_row_bytes = 0, bwd_total = 0, bwd_min = 0;
   long long ldG = 0;
+  // dH = dz . W over the vocabulary: sequential launches of dh_chunk columns, each adding
+  // to dH (dh_kb_part == 0), or one launch split into dh_parts K parts of dh_kb_part
+  // 64-column blocks
+  int dh_chunk = 0, dh_kb_part = 0, dh_parts = 1;
 };
+
+// CTA pairs a launch plans for: a B200 has 148 SMs (the dH split is chosen with it; on
+// another SM count the choice is only less well tuned).
+constexpr int kPlanPairs = 74;
+constexpr int kMaxDhParts = 16;
+
+// Estimated duration of a launch of `units` work units of `kb` K blocks each, in units
+// of one K block on every pair: whole rounds of kPlanPairs units.
+double rounds_x_k(long long units, long long kb) {
+  return static_cast<double>((units + kPlanPairs - 1) / kPlanPairs) * static_cast<double>(kb);
+}
+
+// dH = dz . W has few output tiles (token tiles x column tiles of d), so one launch can
+// leave most of its last wave idle (e.g. 96 tiles on 74 pairs: 2 rounds for 1.3 waves of
+// work). Cutting the vocabulary (K) into parts that run as separate work units of one
+// launch fills the rounds; each part beyond the first costs an fp32 partial sum of the
+// rows (written, then added in part order by a small kernel). A long vocabulary that
+// already fills its rounds keeps sequential launches of kDhVocabChunk columns (measured
+// at the Llama-3.1-8B head: short K loops keep concurrent tiles close in K, so more
+// operand tiles come from L2).
+void plan_dh_split(Plan* p) {
+  const long long kb = (p->V + kBK - 1) / kBK;
+  const long long tiles = static_cast<long long>((p->Nc + 255) / 256) * ((p->d + kBN - 1) / kBN);
+  p->dh_chunk = p->V >= kDhChunkFrom ? kDhVocabChunk : kMaxAccumK;
+  p->dh_kb_part = 0;
+  p->dh_parts = 1;
+  if (p->dtype != DPO_BF16 || tiles == 0 || ((gemm_variant() >> 8) & 1)) return;
+  const double seq = rounds_x_k(tiles, kb);     // one launch or sequential chunks alike
+  if (p->V >= kDhChunkFrom &&
+      static_cast<double>(tiles) / ((tiles + kPlanPairs - 1) / kPlanPairs * kPlanPairs) >= 0.9)
+    return;
+  // the split with the fewest estimated K-block rounds, each extra part charged 2 %
+  const long long max_kbp = kMaxAccumK / kBK;   // K blocks one accumulation may take
+  double best = seq;
+  for (int q = 2; q <= kMaxDhParts; ++q) {
+    long long kbp = (kb + q - 1) / q;
+    if (kbp > max_kbp) continue;
+    const int parts = static_cast<int>((kb + kbp - 1) / kbp);
+    const double est = rounds_x_k(tiles * parts, kbp) * (1.0 + 0.02 * (parts - 1));
+    if (est < best * 0.97) {
+      best = est;
+      p->dh_kb_part = static_cast<int>(kbp);
+      p->dh_parts = parts;
+    }
+  }
+  if (p->dh_parts > 1) {
+    p->dh_chunk = p->V;
+    p->part_row_bytes = static_cast<size_t>(p->dh_parts - 1) * p->d * sizeof(float);
+  }
+}
 
 dpo_status make_plan(const dpo_batch* b, Plan* p) {
   if (b == nullptr) return DPO_ERR_INVALID_ARG;
@@ -190,10 +245,12 @@ dpo_status make_plan(const dpo_batch* b, Plan* p) {
   p->ldG = bf16 ? static_cast<long long>(align_up(b->V, 8)) : b->V;
   p->g_row_bytes = static_cast<size_t>(p->ldG) * (bf16 ? 2 : 4);
   p->off_G = o;
+  plan_dh_split(p);
   const size_t full_rows = Nc > 0 ? Nc : 1;
   const size_t min_rows = full_rows < static_cast<size_t>(kMinChunk) ? full_rows : kMinChunk;
-  p->bwd_total = align_up(o + full_rows * p->g_row_bytes, kAlign);
-  p->bwd_min = align_up(o + min_rows * p->g_row_bytes, kAlign);
+  const size_t row_bytes = p->g_row_bytes + p->part_row_bytes;
+  p->bwd_total = align_up(o + full_rows * row_bytes + kAlign, kAlign);
+  p->bwd_min = align_up(o + min_rows * row_bytes + kAlign, kAlign);
   return DPO_OK;
 }
 
@@ -245,6 +302,9 @@ dpo_status stage_schedule(const Plan& p, const dpo_batch* b, void* ws, const Dev
                                  p.R, p.L, p.d, p.V, p.v0, p.Vtot, p.Nc, Hp, ctl, st));
 }
 
+// Gradient outputs are written 16 bytes at a time (NULL passes: it means "not wanted").
+bool aligned16(const void* ptr) { return reinterpret_cast<uintptr_t>(ptr) % 16 == 0; }
+
 bool ws_ok(const void* ws, size_t have, size_t need) {
   return ws != nullptr && have >= need && reinterpret_cast<uintptr_t>(ws) % kAlign == 0;
 }
@@ -287,17 +347,27 @@ int sm_budget(const DevInfo& di, int max_sms) {
 // Token chunk of the backward that fits the workspace (a multiple of 128 unless it
 // covers every scored position; never more than kMaxAccumK, dW's K per chunk).
 int backward_chunk(const Plan& p, size_t ws_bytes) {
-  const size_t rows_fit = ws_bytes > p.off_G ? (ws_bytes - p.off_G) / p.g_row_bytes : 0;
+  const size_t row_bytes = p.g_row_bytes + p.part_row_bytes;
+  const size_t rows_fit =
+      ws_bytes > p.off_G + kAlign ? (ws_bytes - p.off_G - kAlign) / row_bytes : 0;
   int Mc = static_cast<int>(std::min<size_t>(rows_fit, static_cast<size_t>(p.Nc)));
   Mc = std::min(Mc, kMaxAccumK);
   if (Mc < p.Nc) Mc = Mc / kMinChunk * kMinChunk;
   return Mc;
 }
 
+// Split-K partial sums of a token chunk of mc positions: after its dz rows.
+float* dh_part_scratch(const Plan& p, uint8_t* w, int mc) {
+  if (p.dh_parts < 2) return nullptr;
+  return reinterpret_cast<float*>(w + align_up(p.off_G + static_cast<size_t>(mc) * p.g_row_bytes,
+                                               kAlign));
+}
+
 // dH rows of the packed positions [tok0, tok0 + mc) from the dz chunk in the workspace:
-// dH = dz . W, reduced over the vocabulary in one launch or in chunks of kDhVocabChunk
-// columns for a long vocabulary (never longer than kMaxAccumK), the later chunks added
-// to the rows by the epilogue.
+// dH = dz . W, reduced over the vocabulary in one launch (split into K parts when that
+// fills the GPU's waves better, see plan_dh_split) or in sequential chunks of
+// kDhVocabChunk columns for a long vocabulary, the later chunks added to the rows by
+// the epilogue. No accumulation runs longer than kMaxAccumK products.
 dpo_status run_dh(const Plan& p, const dpo_batch* batch, uint8_t* w, const Sched& sc, int tok0,
                   int mc, float* dH, int sms, const DevCtl& ctl, cudaStream_t st) {
   if (p.dtype != DPO_BF16) {
@@ -306,16 +376,16 @@ dpo_status run_dh(const Plan& p, const dpo_batch* batch, uint8_t* w, const Sched
                                      p.V, dH, st));
   }
   const uint16_t* G = reinterpret_cast<const uint16_t*>(w + p.off_G);
-  const int dh_chunk = p.V >= kDhChunkFrom ? kDhVocabChunk : kMaxAccumK;
-  for (int v0 = 0; v0 < p.V; v0 += dh_chunk) {
-    const int vc = std::min(dh_chunk, p.V - v0);
+  float* part = dh_part_scratch(p, w, mc);
+  for (int v0 = 0; v0 < p.V; v0 += p.dh_chunk) {
+    const int vc = std::min(p.dh_chunk, p.V - v0);
     CUtensorMap mGk, mWmn;
     if (!make_map(&mGk, G + v0, vc, mc, 2ull * p.ldG, kBK, kBoxRows) ||
         !make_map(&mWmn, static_cast<const uint16_t*>(batch->W) + static_cast<size_t>(v0) * p.d,
                   p.d, vc, 2ull * p.d, kBoxMN, kBK))
       return DPO_ERR_CUDA;
-    if (launch_bwd_dh(mGk, mWmn, mc, vc, p.d, tok0, sc.dst, dH, v0 > 0 ? 1 : 0, sms, sc.sync, ctl,
-                      st) != cudaSuccess)
+    if (launch_bwd_dh(mGk, mWmn, mc, vc, p.d, tok0, sc.dst, dH, v0 > 0 ? 1 : 0, part,
+                      p.dh_kb_part, sms, sc.sync, ctl, st) != cudaSuccess)
       return DPO_ERR_CUDA;
   }
   return DPO_OK;
@@ -353,6 +423,7 @@ dpo_status backward_core(const Plan& p, const dpo_batch* batch, const float* lse
                          size_t ws_bytes, void* stream) {
   dpo_status s = DPO_OK;
   if ((p.Nc > 0 && lse_state == nullptr) || row_coef == nullptr) return DPO_ERR_INVALID_ARG;
+  if (!aligned16(dH) || !aligned16(dW)) return DPO_ERR_INVALID_ARG;   // 16-byte row stores
   if (!ws_ok(ws, ws_bytes, p.bwd_min)) return DPO_ERR_WORKSPACE;
   const int Mc = backward_chunk(p, ws_bytes);
   if (p.Nc > 0 && Mc < 1) return DPO_ERR_WORKSPACE;
@@ -582,8 +653,8 @@ dpo_status dpo_backward_dw(const dpo_batch* batch, int32_t v_begin, int32_t v_en
   Plan p;
   dpo_status s = make_plan(batch, &p);
   if (s != DPO_OK) return s;
-  if (dW == nullptr || v_begin < 0 || v_end > p.V || v_begin > v_end || v_begin % 8 != 0 ||
-      (v_end % 8 != 0 && v_end != p.V))
+  if (dW == nullptr || !aligned16(dW) || v_begin < 0 || v_end > p.V || v_begin > v_end ||
+      v_begin % 8 != 0 || (v_end % 8 != 0 && v_end != p.V))
     return DPO_ERR_INVALID_ARG;
   if ((s = dz_resident(p, ws, ws_bytes, max_sms)) != DPO_OK) return s;
   if (v_begin == v_end) return DPO_OK;
@@ -608,7 +679,7 @@ dpo_status dpo_backward_dh(const dpo_batch* batch, float* dH, int32_t max_sms, v
   Plan p;
   dpo_status s = make_plan(batch, &p);
   if (s != DPO_OK) return s;
-  if (dH == nullptr) return DPO_ERR_INVALID_ARG;
+  if (dH == nullptr || !aligned16(dH)) return DPO_ERR_INVALID_ARG;
   if ((s = dz_resident(p, ws, ws_bytes, max_sms)) != DPO_OK) return s;
   DevInfo di;
   if ((s = device_info(&di)) != DPO_OK) return s;
@@ -688,7 +759,7 @@ dpo_status dpo_selftest_wait_timeout(uint32_t budget_ms, void* stream) {
 }
 
 int32_t dpo_set_gemm_variant(int32_t variant) {
-  if (variant < 0 || variant > 255) return -1;
+  if (variant < 0 || variant > 511) return -1;
   return g_gemm_variant.exchange(variant);
 }
 

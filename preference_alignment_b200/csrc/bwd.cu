@@ -42,7 +42,8 @@ struct EpiGrad {
   float nl2, cf;
   EpiCtx ctx;
 
-  __device__ __forceinline__ void begin(const Params& p, int m_row, int nt, const EpiCtx& c) {
+  __device__ __forceinline__ void begin(const Params& p, int m_row, int nt, int,
+                                        const EpiCtx& c) {
     const int tok = m_row;
     ctx = c;
     row0 = tok - c.lane;                 // first row of this warp's 32-row block
@@ -98,23 +99,36 @@ struct EpiGrad {
 };
 
 // ------------------------------------------------------------------ dH rows epilogue
+// K part 0 of a unit writes (or adds to) the dH rows of its positions; with split-K
+// the later parts write their partial sums to fp32 scratch, which k_dh_reduce adds
+// to the rows in part order.
 struct EpiRows {
   static constexpr bool kStaging = false;   // stores go straight to global memory
   struct Params {
     const int* dst;        // packed position -> flat row r * L + t
     float* out;            // dH [R * L, d]
+    float* part;           // split-K scratch [k_parts - 1, Mc, d] of parts 1.. (or null)
     int Mc, d, tok0;
-    int accumulate;        // 1: add to the rows (later vocabulary chunks of K)
+    int accumulate;        // part 0 adds to the rows (a later vocabulary chunk of K)
   };
   float* o;
   int nbase;
-  bool valid;
+  bool valid, acc;
 
-  __device__ __forceinline__ void begin(const Params& p, int m_row, int nt, const EpiCtx&) {
+  __device__ __forceinline__ void begin(const Params& p, int m_row, int nt, int ks,
+                                        const EpiCtx&) {
     const int tok = m_row;
     valid = tok < p.Mc;
     nbase = nt * kBN;
-    o = valid ? p.out + static_cast<long long>(__ldg(p.dst + p.tok0 + tok)) * p.d : nullptr;
+    o = nullptr;
+    acc = false;
+    if (!valid) return;
+    if (ks == 0) {
+      o = p.out + static_cast<long long>(__ldg(p.dst + p.tok0 + tok)) * p.d;
+      acc = p.accumulate != 0;
+    } else {
+      o = p.part + (static_cast<long long>(ks - 1) * p.Mc + tok) * p.d;
+    }
   }
 
   __device__ __forceinline__ void chunk(const Params& p, int c, const uint32_t (&v)[32]) {
@@ -126,7 +140,7 @@ struct EpiRows {
         float4 r = make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
                                __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
         float4* dst = reinterpret_cast<float4*>(o + col);
-        if (p.accumulate) {
+        if (acc) {
           const float4 old = *dst;
           r.x += old.x;
           r.y += old.y;
@@ -141,6 +155,31 @@ struct EpiRows {
   __device__ __forceinline__ void end(const Params&) {}
 };
 
+// dH[dst[tok0 + i]] += part[0][i] + part[1][i] + ... (parts in order, one thread per 4
+// columns): the split-K partial sums of K parts 1.., after part 0 wrote the rows.
+__global__ void __launch_bounds__(256) k_dh_reduce(float* __restrict__ dH,
+                                                   const float* __restrict__ part,
+                                                   const int* __restrict__ dst, int tok0, int Mc,
+                                                   int d, int n_extra) {
+  const int d4 = d / 4;
+  const long long q = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (q >= static_cast<long long>(Mc) * d4) return;
+  const int i = static_cast<int>(q / d4);
+  const int c = static_cast<int>(q - static_cast<long long>(i) * d4);
+  float4* o = reinterpret_cast<float4*>(dH + static_cast<long long>(__ldg(dst + tok0 + i)) * d) + c;
+  float4 a = *o;
+  const long long stride = static_cast<long long>(Mc) * d4;
+  const float4* src = reinterpret_cast<const float4*>(part) + q;
+  for (int s = 0; s < n_extra; ++s) {
+    const float4 b = __ldg(src + s * stride);
+    a.x += b.x;
+    a.y += b.y;
+    a.z += b.z;
+    a.w += b.w;
+  }
+  *o = a;
+}
+
 // ------------------------------------------------------------------ dW epilogue
 struct EpiDW {
   static constexpr bool kStaging = false;   // stores go straight to global memory
@@ -152,7 +191,8 @@ struct EpiDW {
   int nbase;
   bool valid;
 
-  __device__ __forceinline__ void begin(const Params& p, int m_row, int nt, const EpiCtx&) {
+  __device__ __forceinline__ void begin(const Params& p, int m_row, int nt, int,
+                                        const EpiCtx&) {
     const int v = m_row;
     valid = v < p.V;
     nbase = nt * kBN;
@@ -189,17 +229,25 @@ cudaError_t launch_bwd_grad(const CUtensorMap& mapA, const CUtensorMap& mapB,
                             int* sync, const DevCtl& ctl, cudaStream_t st) {
   EpiGrad::Params p{y, lse, coef, rowid, Mc, V, tok0};
   return launch_gemm<false, false, EpiGrad>(mapA, mapB, mapG, Mc, V, d, 2, p, grid, ctl, st,
-                                            kGemmGrad, token_group(d), DPO_EPOCH_KB, sync,
-                                            kSyncInts);
+                                            kGemmGrad, token_group(d), sync);
 }
 
 cudaError_t launch_bwd_dh(const CUtensorMap& mapA, const CUtensorMap& mapB, int Mc, int V, int d,
-                          int tok0, const int* dst, float* dH, int accumulate, int grid, int* sync,
-                          const DevCtl& ctl, cudaStream_t st) {
-  EpiRows::Params p{dst, dH, Mc, d, tok0, accumulate};
-  return launch_gemm<false, true, EpiRows>(mapA, mapB, mapA, Mc, d, V, DPO_GROUP_DH > 0 ? 3 : 1, p,
-                                           grid, ctl, st, kGemmDH, DPO_GROUP_DH, DPO_EPOCH_KB,
-                                           sync, kSyncInts);
+                          int tok0, const int* dst, float* dH, int accumulate, float* part,
+                          int kb_part, int grid, int* sync, const DevCtl& ctl, cudaStream_t st) {
+  const int k_blocks = (V + kBK - 1) / kBK;
+  if (kb_part <= 0 || kb_part > k_blocks) kb_part = k_blocks;
+  const int n_extra = split_k_parts(k_blocks, kb_part) - 1;
+  if (n_extra > 0 && (part == nullptr || accumulate)) return cudaErrorInvalidValue;
+  EpiRows::Params p{dst, dH, part, Mc, d, tok0, accumulate};
+  cudaError_t e = launch_gemm<false, true, EpiRows>(mapA, mapB, mapA, Mc, d, V,
+                                                    DPO_GROUP_DH > 0 ? 3 : 1, p, grid, ctl, st,
+                                                    kGemmDH, DPO_GROUP_DH, sync, kb_part);
+  if (e != cudaSuccess || n_extra == 0) return e;
+  const long long n4 = static_cast<long long>(Mc) * (d / 4);
+  k_dh_reduce<<<static_cast<unsigned>((n4 + 255) / 256), 256, 0, st>>>(dH, part, dst, tok0, Mc, d,
+                                                                       n_extra);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_bwd_dw(const CUtensorMap& mapA, const CUtensorMap& mapB, int Mc, int V, int d,
@@ -207,8 +255,7 @@ cudaError_t launch_bwd_dw(const CUtensorMap& mapA, const CUtensorMap& mapB, int 
                           cudaStream_t st) {
   EpiDW::Params p{dW, V, d, accumulate};
   return launch_gemm<true, true, EpiDW>(mapA, mapB, mapA, V, d, Mc, DPO_GROUP_DW > 0 ? 3 : 1, p, grid,
-                                         ctl, st, kGemmDW, DPO_GROUP_DW, DPO_EPOCH_KB, sync,
-                                         kSyncInts);
+                                         ctl, st, kGemmDW, DPO_GROUP_DW, sync);
 }
 
 }  // namespace dpo

@@ -93,7 +93,8 @@ struct EpiLSE {
   bool valid;
   float mx, s, zyv;
 
-  __device__ __forceinline__ void begin(const Params& p, int m_row, int nt_, const EpiCtx&) {
+  __device__ __forceinline__ void begin(const Params& p, int m_row, int nt_, int,
+                                        const EpiCtx&) {
     nt = nt_;
     tok = m_row;
     valid = tok < p.Nc;
@@ -147,8 +148,7 @@ cudaError_t launch_fwd_lse(const CUtensorMap& mapA, const CUtensorMap& mapB, int
   // order 0: all token tiles of one vocab tile run together, so each W tile is
   // read from HBM once and served to the other CTAs from L2
   return launch_gemm<false, false, EpiLSE>(mapA, mapB, mapA, Nc, V, d, 2, p, grid, ctl, st,
-                                           kGemmForward, token_group(d), DPO_EPOCH_KB, sync,
-                                           kSyncInts);
+                                           kGemmForward, token_group(d), sync);
 }
 
 // ------------------------------------------------------------------ combine

@@ -47,31 +47,41 @@ inline double tile_fill(int M, int tile_m, int n_tiles, int slots) {
   return static_cast<double>(M) * n_tiles / (static_cast<double>(waves) * slots * tile_m);
 }
 
+// Number of K parts of kb_part blocks each (the last may be shorter, none is empty).
+inline int split_k_parts(int k_blocks, int kb_part) { return (k_blocks + kb_part - 1) / kb_part; }
+
 // A CTA pair does a 256-row tile ~3 % faster than two single CTAs do its halves
 // (measured under the power cap); the single-CTA kernel is chosen only when its
 // finer tiles fill the GPU's waves better by more than this margin.
 constexpr double kPairMargin = 1.05;
 
-// D[M x N] = A[M x K] . B[N x K]^T with the epilogue Epi; `order` picks the tile
-// raster (0: M fastest, 1: N fastest); `sms` is the device's SM count.
-// Raster: `order` as in GemmGeom (0, 1, or 2/3 grouped along M/N with `group`
-// 256-wide tiles per group; a group of 0 falls back to order 0).
-// `kind` (a GemmKind) selects this GEMM's bit of the dpo_set_gemm_variant mask: a set
-// bit forces the single-CTA kernel; a clear bit runs CTA pairs unless 128-row tiles
-// fill the waves clearly better (tile_fill), e.g. 4,648 rows x 8 column tiles: 152
-// pair tiles are 2.05 waves of 74 pairs (3 launched, 68 % full), 296 single tiles
-// exactly 2 waves of 148 CTAs.
+// D[M x N] = A[M x K] . B[N x K]^T with the epilogue Epi; `sms` is the device's SM
+// count (or the SM budget of this launch).
+// Raster: `order` as in GemmGeom (0: M fastest, 1: N fastest, 2/3 grouped along M/N
+// with `group` 256-wide tiles per group; a group of 0 falls back to order 0).
+// `kind` (a GemmKind) selects this GEMM's bits of the dpo_set_gemm_variant mask:
+//   bit kind      set: the single-CTA kernel; clear: CTA pairs unless 128-row tiles
+//                 fill the waves clearly better (tile_fill), e.g. 4,648 rows x 8 column
+//                 tiles: 152 pair tiles are 2.05 waves of 74 pairs (3 launched, 68 %
+//                 full), 296 single tiles exactly 2 waves of 148 CTAs;
+//   bit 4 + kind  set: the pair kernel's static tile schedule; clear: tiles claimed in
+//                 raster order from `counter` (one int of workspace, zeroed here).
 // mapC is the epilogue's store tensor map (epilogues that do not store through TMA
 // ignore it; pass any valid map).
+// kb_part > 0 splits K into parts of kb_part K blocks (split_k_parts gives their
+// count); each part of a tile is its own work unit and the epilogue learns its part.
 template <bool A_MN, bool B_MN, class Epi>
 cudaError_t launch_gemm(const CUtensorMap& mapA, const CUtensorMap& mapB, const CUtensorMap& mapC,
                         int M, int N, int K, int order, const typename Epi::Params& p, int sms,
-                        const DevCtl& ctl, cudaStream_t st, int kind, int group = 0,
-                        int epoch = 0, int* sync = nullptr, int sync_len = 0) {
+                        const DevCtl& ctl, cudaStream_t st, int kind, int group, int* counter,
+                        int kb_part = 0) {
   if (order >= 2 && group <= 0) order = 0;
   const int n_tiles = (N + kBN - 1) / kBN;
   const int k_blocks = (K + kBK - 1) / kBK;
-  if (((gemm_variant() >> kind) & 1) == 0) {
+  if (kb_part <= 0 || kb_part > k_blocks) kb_part = k_blocks;
+  const int k_parts = split_k_parts(k_blocks, kb_part);
+  const int variant = gemm_variant();
+  if (((variant >> kind) & 1) == 0) {
     auto kern = k_tc_gemm_pair<A_MN, B_MN, Epi>;
     constexpr int smem = pair_smem_bytes<Epi>();
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -79,23 +89,19 @@ cudaError_t launch_gemm(const CUtensorMap& mapA, const CUtensorMap& mapB, const 
     const int clusters = max_pair_clusters(kern, smem);
     if (clusters > 0) {
       GemmGeom g{(M + kPairM - 1) / kPairM, n_tiles, k_blocks, order, group > 0 ? group : 1,
-                 0, nullptr};
-      const int tiles = g.m_tiles * g.n_tiles;
+                 k_parts, kb_part, nullptr};
+      const int tiles = g.m_tiles * g.n_tiles * k_parts;
       int pairs = clusters < sms / 2 ? clusters : sms / 2;
       if (pairs > tiles) pairs = tiles;
       if (pairs < 1) pairs = 1;
       const bool single_fills_better =
-          tile_fill(M, kBM, n_tiles, sms) > kPairMargin * tile_fill(M, kPairM, n_tiles, pairs);
+          tile_fill(M, kBM, n_tiles * k_parts, sms) >
+          kPairMargin * tile_fill(M, kPairM, n_tiles * k_parts, pairs);
       if (!single_fills_better) {
-        if (epoch > 0 && sync != nullptr) {
-          // epochs this launch can reach; pacing stays off if the counters do not fit
-          const long long per_pair = static_cast<long long>((tiles + pairs - 1) / pairs) * k_blocks;
-          if (per_pair / epoch + 1 < sync_len) {
-            e = cudaMemsetAsync(sync, 0, sizeof(int) * (per_pair / epoch + 2), st);
-            if (e != cudaSuccess) return e;
-            g.epoch = epoch;
-            g.sync = sync;
-          }
+        if (((variant >> (4 + kind)) & 1) == 0 && counter != nullptr) {
+          e = cudaMemsetAsync(counter, 0, sizeof(int), st);
+          if (e != cudaSuccess) return e;
+          g.counter = counter;
         }
         kern<<<2 * pairs, kGemmThreads, smem, st>>>(mapA, mapB, mapC, g, p, ctl);
         return cudaGetLastError();
@@ -107,8 +113,8 @@ cudaError_t launch_gemm(const CUtensorMap& mapA, const CUtensorMap& mapB, const 
                                        kGemmSmemBytes);
   if (e != cudaSuccess) return e;
   GemmGeom g{(M + kBM - 1) / kBM, n_tiles, k_blocks, order,
-             group > 0 ? (order == 2 ? 2 * group : group) : 1, 0, nullptr};
-  const int tiles = g.m_tiles * g.n_tiles;
+             group > 0 ? (order == 2 ? 2 * group : group) : 1, k_parts, kb_part, nullptr};
+  const int tiles = g.m_tiles * g.n_tiles * k_parts;
   kern<<<sms < tiles ? sms : tiles, kGemmThreads, kGemmSmemBytes, st>>>(mapA, mapB, mapC, g, p,
                                                                         ctl);
   return cudaGetLastError();

@@ -95,10 +95,14 @@ cudaError_t launch_bwd_grad(const CUtensorMap& mapA, const CUtensorMap& mapB,
                             const float* lse, const float* coef, const int* rowid, int grid,
                             int* sync, const DevCtl& ctl, cudaStream_t st);
 
-// dH rows: out[dst[tok0 + i]] = (G . W)[i]   (A = G K-major, B = W MN-major)
+// dH rows: out[dst[tok0 + i]] (+)= (G . W)[i]   (A = G K-major, B = W MN-major)
+// kb_part > 0 splits K (the vocabulary) into parts of kb_part 64-column blocks run as
+// separate work units of one launch; parts 1.. write fp32 partial sums to `part`
+// ([parts - 1, Mc, d]) and a reduce kernel adds them to the rows in part order
+// (split-K needs accumulate == 0).
 cudaError_t launch_bwd_dh(const CUtensorMap& mapA, const CUtensorMap& mapB, int Mc, int V, int d,
-                          int tok0, const int* dst, float* dH, int accumulate, int grid, int* sync,
-                          const DevCtl& ctl, cudaStream_t st);
+                          int tok0, const int* dst, float* dH, int accumulate, float* part,
+                          int kb_part, int grid, int* sync, const DevCtl& ctl, cudaStream_t st);
 
 // dW (+)= G^T . Hp   (A = G MN-major, B = Hp MN-major)
 cudaError_t launch_bwd_dw(const CUtensorMap& mapA, const CUtensorMap& mapB, int Mc, int V, int d,

@@ -55,33 +55,17 @@ struct GemmGeom {
   int m_tiles, n_tiles, k_blocks;
   int order;
   int group;
-  // Optional pacing of the CTA pairs (0 = off): every `epoch` K blocks the leader
-  // producers meet at a counter in `sync` (sync[0] counts pairs that have finished,
-  // sync[1 + e] pairs past epoch e), so concurrent tiles stay within about two
-  // epochs of each other and keep sharing the operand lines in L2.
-  int epoch;
-  int* sync;
+  // Split-K: the K blocks are cut into k_parts parts of kb_part blocks (the last may be
+  // shorter, none empty); a work unit is (part, m tile, n tile), parts outermost, and
+  // the epilogue learns its part. k_parts = 1: one unit per output tile.
+  int k_parts, kb_part;
+  // Tile claim counter of the CTA-pair kernel (zeroed before the launch), or nullptr
+  // for the static schedule (pair p takes tiles p, p + n_pairs, ...). With the counter
+  // each pair claims its next tile in raster order when it starts loading it, so the
+  // tiles in flight stay one contiguous window of the raster even when pairs run at
+  // different speeds, and share their operand tiles in L2.
+  int* counter;
 };
-
-// A leader producer that has finished epoch e records it, then waits (bounded) until
-// every pair has finished epoch e - 1 (or has no work left). The one epoch of slack
-// keeps the fast pairs issuing loads while the slow ones catch up, and still bounds
-// the distance between any two pairs to about two epochs.
-__device__ __forceinline__ bool pace_epoch(const GemmGeom& g, int e, int n_pairs,
-                                           const DevCtl& ctl, volatile int* abort_flag) {
-  atomicAdd(g.sync + 1 + e, 1);
-  if (e == 0) return true;
-  const unsigned long long t0 = globaltimer_ns();
-  while (true) {
-    int a, f;
-    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(a) : "l"(g.sync + e) : "memory");
-    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(f) : "l"(g.sync) : "memory");
-    if (a + f >= n_pairs) return true;
-    if (*abort_flag) return false;
-    if (globaltimer_ns() - t0 > ctl.budget_ns) return false;
-    __nanosleep(64);
-  }
-}
 
 __device__ __forceinline__ void tile_coords(const GemmGeom& g, int tile, int& mt, int& nt) {
   if (g.order == 0) {
@@ -111,9 +95,20 @@ __device__ __forceinline__ void tile_coords(const GemmGeom& g, int tile, int& mt
   }
 }
 
-// Epilogue interface (one object per epilogue thread, per tile; every thread of the
+// Work unit -> K part ks, tile (mt, nt) and the unit's K blocks [kb0, kb1).
+__device__ __forceinline__ void unit_coords(const GemmGeom& g, int unit, int& ks, int& mt, int& nt,
+                                            int& kb0, int& kb1) {
+  const int per_part = g.m_tiles * g.n_tiles;
+  ks = unit / per_part;
+  tile_coords(g, unit - ks * per_part, mt, nt);
+  kb0 = ks * g.kb_part;
+  kb1 = min(g.k_blocks, kb0 + g.kb_part);
+}
+
+// Epilogue interface (one object per epilogue thread, per unit; every thread of the
 // warp calls each method, in step):
-//   __device__ void begin(const Params&, int m_row, int nt, const EpiCtx&);   // m_row: row of D
+//   __device__ void begin(const Params&, int m_row, int nt, int ks, const EpiCtx&);
+//       m_row: row of D; nt: column tile; ks: K part of the unit (0 without split-K)
 //   __device__ void chunk(const Params&, int c, const uint32_t (&v)[32]);   // columns c*32..+31
 //   __device__ void end(const Params&);
 template <bool A_MN, bool B_MN, class Epi>
@@ -168,7 +163,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  const int n_tiles_total = g.m_tiles * g.n_tiles;
+  const int n_tiles_total = g.m_tiles * g.n_tiles * g.k_parts;   // work units
   // Producer bookkeeping kept for the teardown: which stages have a load issued
   // and the parity of the `full` phase that load completes.
   uint32_t issued_mask = 0, issued_par = 0;
@@ -179,9 +174,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint32_t phase = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < n_tiles_total && ok; tile += gridDim.x) {
-      int mt, nt;
-      tile_coords(g, tile, mt, nt);
-      for (int kb = 0; kb < g.k_blocks; ++kb) {
+      int ks, mt, nt, kb0, kb1;
+      unit_coords(g, tile, ks, mt, nt, kb0, kb1);
+      for (int kb = kb0; kb < kb1; ++kb) {
         if (!mbar_wait(empty0 + 8 * stage, phase ^ 1, ctl, abort_flag)) {
           ok = false;
           break;
@@ -234,7 +229,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + acc * kBN;
-      for (int kb = 0; kb < g.k_blocks; ++kb) {
+      int ks, mt, nt, kb0, kb1;
+      unit_coords(g, tile, ks, mt, nt, kb0, kb1);
+      for (int kb = kb0; kb < kb1; ++kb) {
         if (!mbar_wait(full0 + 8 * stage, phase, ctl, abort_flag)) {
           ok = false;
           break;
@@ -250,7 +247,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                    : sw128_desc(a0 + k * 32, 16, 1024);
           const uint64_t bd = B_MN ? sw128_desc(b0 + k * 2048, 8192, 1024)
                                    : sw128_desc(b0 + k * 32, 16, 1024);
-          tc_mma_f16(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
+          tc_mma_f16(d_tmem, ad, bd, idesc, (kb != kb0 || k != 0) ? 1u : 0u);
         }
         tc_commit(empty0 + 8 * stage);   // frees this stage once its MMAs are done
         if (++stage == kStages) {
@@ -287,10 +284,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         break;
       }
       tc_fence_after();
-      int mt, nt;
-      tile_coords(g, tile, mt, nt);
+      int ks, mt, nt, kb0, kb1;
+      unit_coords(g, tile, ks, mt, nt, kb0, kb1);
       Epi epi;
-      epi.begin(ep, mt * kBM + row, nt, ectx);
+      epi.begin(ep, mt * kBM + row, nt, ks, ectx);
 #pragma unroll 1
       for (int c = 0; c < kBN / 32; ++c) {
         uint32_t v[32];
@@ -353,10 +350,35 @@ constexpr int kPStageBytes = kPABytes + kPBBytes;
 // 6 stages were 0.2-2.3 % faster.
 template <class Epi>
 constexpr int pair_stages() { return 6; }
+// Schedule ring of the dynamic tile schedule: slots of claimed tile indices, written
+// by the leader's producer into both CTAs and read by every role.
+constexpr int kSchedSlots = 4;
+// Readers of a slot, each arriving once on the leader's `sched_empty`: the follower's
+// producer, the leader's MMA issuer and the 4 epilogue warps of each CTA.
+constexpr int kSchedReaders = 1 + 1 + 2 * 4;
 template <class Epi>
 constexpr int pair_smem_bytes() {
-  return pair_stages<Epi>() * kPStageBytes + (Epi::kStaging ? kEpiSmemBytes : 0) + 1024 + 256;
+  return pair_stages<Epi>() * kPStageBytes + (Epi::kStaging ? kEpiSmemBytes : 0) + 1024 + 512;
 }
+
+// The schedule ring as one role sees it: slot i holds the pair's i-th tile (-1 = none
+// left). `full` barriers live in each CTA (one release-arrive from the leader's
+// producer per phase); `empty` barriers are the leader's.
+struct SchedRing {
+  uint32_t full0, empty_leader0, tile0;   // shared addresses (empty: shared::cluster)
+
+  // A reader takes slot i: wait (bounded, cluster-scope acquire) until it is published,
+  // read the tile, release the slot to the leader. False when the wait gave up.
+  __device__ __forceinline__ bool take(int i, int& tile, const DevCtl& ctl,
+                                       volatile int* abort_flag) const {
+    const int slot = i % kSchedSlots;
+    const uint32_t ph = static_cast<uint32_t>(i / kSchedSlots) & 1u;
+    if (!mbar_wait_cluster(full0 + 8 * slot, ph, ctl, abort_flag)) return false;
+    tile = static_cast<int>(ld_shared_u32(tile0 + 4 * slot));
+    mbar_arrive_cluster(empty_leader0 + 8 * slot);
+    return true;
+  }
+};
 
 template <bool A_MN, bool B_MN, class Epi>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
@@ -372,7 +394,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   uint8_t* sB = smem + kPStages * kPABytes;
   uint8_t* sE = smem + kPStages * kPStageBytes;        // epilogue staging (Epi::kStaging)
   uint64_t* bars = reinterpret_cast<uint64_t*>(sE + (Epi::kStaging ? kEpiSmemBytes : 0));
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kPStages + 5);
+  // bars: [0, S) full, [S, 2S) empty, 2S + {0,1} acc_full, 2S + {2,3} acc_empty,
+  // 2S + 4 drain, then kSchedSlots sched_full and kSchedSlots sched_empty
+  int* sched_tile = reinterpret_cast<int*>(bars + 2 * kPStages + 5 + 2 * kSchedSlots);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sched_tile + kSchedSlots);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -384,6 +409,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   const uint32_t accf0 = smem_u32(bars + 2 * kPStages);
   const uint32_t acce0 = smem_u32(bars + 2 * kPStages + 2);
   const uint32_t drain = smem_u32(bars + 2 * kPStages + 4);
+  const uint32_t sfull0 = smem_u32(bars + 2 * kPStages + 5);
+  const uint32_t sempty0 = smem_u32(bars + 2 * kPStages + 5 + kSchedSlots);
+  const SchedRing ring{sfull0, mapa_shared(sempty0, 0), smem_u32(sched_tile)};
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kPStages; ++s) {
@@ -395,6 +423,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       mbar_init(acce0 + 8 * a, 2 * 128);    // leader: every epilogue thread of both CTAs
     }
     mbar_init(drain, 1);
+    for (int s = 0; s < kSchedSlots; ++s) {
+      mbar_init(sfull0 + 8 * s, 1);         // the leader producer's release-arrive
+      mbar_init(sempty0 + 8 * s, kSchedReaders);
+    }
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
@@ -411,27 +443,46 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 
   const int pair = blockIdx.x >> 1;
   const int n_pairs = gridDim.x >> 1;
-  const int n_tiles_total = g.m_tiles * g.n_tiles;   // m_tiles counts 256-row tiles
+  const int n_tiles_total = g.m_tiles * g.n_tiles * g.k_parts;   // work units (256-row tiles)
+  const bool dyn = g.counter != nullptr;
 
   if (warp == 0 && lane == 0) {
     // ---------------------------------------------------------------- TMA producer
+    // (the leader's also claims the pair's tiles and publishes them in the ring)
     const uint32_t full_leader = mapa_shared(full0, 0);
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
-    long long gk = 0;                       // K blocks issued by this pair so far
-    const bool pacer = leader && g.epoch > 0;
-    for (int tile = pair; tile < n_tiles_total && ok; tile += n_pairs) {
-      int mt, nt;
-      tile_coords(g, tile, mt, nt);
-      const int arow = mt * kPairM + static_cast<int>(rank) * 128;
-      const int brow = nt * kBN + static_cast<int>(rank) * (kBN / 2);
-      for (int kb = 0; kb < g.k_blocks; ++kb, ++gk) {
-        if (pacer && gk > 0 && gk % g.epoch == 0 &&
-            !pace_epoch(g, static_cast<int>(gk / g.epoch) - 1, n_pairs, ctl, abort_flag)) {
+    for (int i = 0; ok; ++i) {
+      int tile = pair + i * n_pairs;
+      if (dyn) {
+        if (leader) {
+          const int slot = i % kSchedSlots;
+          const uint32_t ph = static_cast<uint32_t>(i / kSchedSlots) & 1u;
+          if (!mbar_wait(sempty0 + 8 * slot, ph ^ 1u, ctl, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tile = atomicAdd(g.counter, 1);
+          if (tile >= n_tiles_total) tile = -1;
+          for (uint32_t r = 0; r < 2; ++r) {
+            st_shared_cluster_u32(mapa_shared(ring.tile0 + 4 * slot, r),
+                                  static_cast<uint32_t>(tile));
+            mbar_arrive_cluster(mapa_shared(sfull0 + 8 * slot, r));
+          }
+        } else if (!ring.take(i, tile, ctl, abort_flag)) {
           ok = false;
           break;
         }
+        if (tile < 0) break;
+      } else if (tile >= n_tiles_total) {
+        break;
+      }
+      int ks, mt, nt, kb0, kb1;
+      unit_coords(g, tile, ks, mt, nt, kb0, kb1);
+      const int arow = mt * kPairM + static_cast<int>(rank) * 128;
+      const int brow = nt * kBN + static_cast<int>(rank) * (kBN / 2);
+      for (int kb = kb0; kb < kb1; ++kb) {
         if (!mbar_wait(empty0 + 8 * stage, phase ^ 1, ctl, abort_flag)) {
           ok = false;
           break;
@@ -458,7 +509,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         }
       }
     }
-    if (pacer) atomicAdd(g.sync, 1);        // finished: count as arrived at every later epoch
     if (!ok) {
       record_status(ctl, kStatusTimeout);
       *abort_flag = 1;
@@ -470,7 +520,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     uint32_t phase = 0;
     int local = 0;
     bool ok = true;
-    for (int tile = pair; tile < n_tiles_total && ok; tile += n_pairs, ++local) {
+    for (int i = 0; ok; ++i, ++local) {
+      int tile = pair + i * n_pairs;
+      if (dyn) {
+        if (!ring.take(i, tile, ctl, abort_flag)) {
+          ok = false;
+          break;
+        }
+        if (tile < 0) break;
+      } else if (tile >= n_tiles_total) {
+        break;
+      }
       const int acc = local & 1;
       const uint32_t acc_phase = (local >> 1) & 1;
       if (!mbar_wait(acce0 + 8 * acc, acc_phase ^ 1, ctl, abort_flag)) {
@@ -479,7 +539,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       }
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + acc * kBN;
-      for (int kb = 0; kb < g.k_blocks; ++kb) {
+      int ks, mt, nt, kb0, kb1;
+      unit_coords(g, tile, ks, mt, nt, kb0, kb1);
+      for (int kb = kb0; kb < kb1; ++kb) {
         if (!mbar_wait(full0 + 8 * stage, phase, ctl, abort_flag)) {
           ok = false;
           break;
@@ -493,7 +555,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                                    : sw128_desc(a0 + k * 32, 16, 1024);
           const uint64_t bd = B_MN ? sw128_desc(b0 + k * 2048, 8192, 1024)
                                    : sw128_desc(b0 + k * 32, 16, 1024);
-          tc_mma_f16_pair(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
+          tc_mma_f16_pair(d_tmem, ad, bd, idesc, (kb != kb0 || k != 0) ? 1u : 0u);
         }
         tc_commit_pair_mc(empty0 + 8 * stage, 0x3);
         if (++stage == kPStages) {
@@ -519,7 +581,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     const uint32_t acce_leader = mapa_shared(acce0, 0);
     const EpiCtx ectx{&tmC, smem_u32(sE + (warp - 2) * kEpiWarpBytes), lane};
     int local = 0;
-    for (int tile = pair; tile < n_tiles_total; tile += n_pairs, ++local) {
+    for (int i = 0;; ++i, ++local) {
+      int tile = pair + i * n_pairs;
+      if (dyn) {
+        // lane 0 takes the slot for the warp (one release per warp) and shares the tile
+        int ok = 1;
+        if (lane == 0) ok = ring.take(i, tile, ctl, abort_flag) ? 1 : 0;
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        tile = __shfl_sync(0xffffffffu, tile, 0);
+        if (!ok) {
+          if (lane == 0) {
+            record_status(ctl, kStatusTimeout);
+            *abort_flag = 1;
+          }
+          break;
+        }
+        if (tile < 0) break;
+      } else if (tile >= n_tiles_total) {
+        break;
+      }
       const int acc = local & 1;
       const uint32_t acc_phase = (local >> 1) & 1;
       if (!mbar_wait(accf0 + 8 * acc, acc_phase, ctl, abort_flag)) {
@@ -528,10 +608,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         break;
       }
       tc_fence_after();
-      int mt, nt;
-      tile_coords(g, tile, mt, nt);
+      int ks, mt, nt, kb0, kb1;
+      unit_coords(g, tile, ks, mt, nt, kb0, kb1);
       Epi epi;
-      epi.begin(ep, mt * kPairM + row, nt, ectx);
+      epi.begin(ep, mt * kPairM + row, nt, ks, ectx);
 #pragma unroll 1
       for (int c = 0; c < kBN / 32; ++c) {
         uint32_t v[32];

@@ -26,15 +26,8 @@ constexpr int kBoxMN = 64;     // columns of an MN-major TMA box (one 128-byte s
 #ifndef DPO_GROUP_DW
 #define DPO_GROUP_DW 0
 #endif
-// Pacing of the CTA pairs inside a GEMM (K blocks per epoch, 0 = off) and the
-// size of the workspace counter area it uses. Measured at the Llama-3.1-8B head:
-// with 64-block epochs the DRAM reads per launch fall (forward 6.1 -> 2.5 GB, dH
-// 29 -> 12.7 GB, dW 20.8 -> 12.3 GB) because concurrent tiles stay in step and
-// share L2 lines, but the waiting costs as much time as the traffic saves, so the
-// default is off.
-#ifndef DPO_EPOCH_KB
-#define DPO_EPOCH_KB 0
-#endif
-constexpr int kSyncInts = 16384;
+// Ints of the workspace's counter area (the pair kernels' tile claim counter is the
+// first; each GEMM launch zeroes it before it starts).
+constexpr int kSyncInts = 64;
 
 }  // namespace dpo

@@ -316,7 +316,8 @@ def fingerprint(data, nbytes, out, stream=None):
 
 def set_gemm_variant(variant: int) -> int:
     """Mask per GEMM k (forward, dz, dH, dW): bit k runs it on the single-CTA kernel, bit 4 + k
-    gives the CTA-pair kernel the static tile schedule instead of tiles claimed in raster order."""
+    gives the CTA-pair kernel the static tile schedule instead of tiles claimed in raster order;
+    bit 8 keeps dH from being split over the vocabulary (set it before sizing workspaces)."""
     lib = load()
     fn = lib.dpo_set_gemm_variant
     fn.argtypes = [ctypes.c_int32]

@@ -112,6 +112,12 @@ def test_calls_fail_on_the_host_and_leave_outputs_alone(lib):
     with pytest.raises(libdpo.DpoError) as e:   # backward without row coefficients
         libdpo.backward(b, FAKE, None, None, FAKE, False, FAKE, ws_bytes=1 << 30)
     assert e.value.status == libdpo.ERR_INVALID_ARG
+    with pytest.raises(libdpo.DpoError) as e:   # dW not 16-byte aligned
+        libdpo.backward(b, FAKE, FAKE, None, FAKE + 4, False, FAKE, ws_bytes=1 << 30)
+    assert e.value.status == libdpo.ERR_INVALID_ARG
+    with pytest.raises(libdpo.DpoError) as e:   # dH not 16-byte aligned
+        libdpo.backward(b, FAKE, FAKE, FAKE + 8, FAKE, False, FAKE, ws_bytes=1 << 30)
+    assert e.value.status == libdpo.ERR_INVALID_ARG
     bl = _batch(L=128, C=[100, 100, 100, 100])    # 400 scored positions: chunked below bwd
     _, bwl, mnl = libdpo.workspace_size(bl)
     assert mnl < bwl

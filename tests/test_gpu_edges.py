@@ -151,22 +151,29 @@ def test_single_cta_gemm_kernel(shape):
 
 
 def test_gemm_variants_agree():
+    """Single-CTA and CTA-pair kernels, and dH with or without split-K (0x100), agree
+    within rounding; the pair kernel's two tile schedules (claimed in raster order, or
+    static round-robin: 0xF0) compute every tile the same way, so they agree bit for bit."""
     import torch
     w = WL.make_custom(R=4, L=400, d=256, V=1500, dtype="bf16", seed=91, prompt_range=(1, 100))
     dw = DeviceWorkload(w)
     outs = []
-    for v in (0, 15, 5):
+    for v in (0, 15, 5, 0x100, 0xF0, 0x50):
         old = libdpo.set_gemm_variant(v)
         try:
             seq, tok, lse = dw.forward(dw.W, want_grad=True)
             dH, dW = dw.backward(lse, torch.linspace(-0.1, 0.1, 4, device="cuda"))
         finally:
             libdpo.set_gemm_variant(old)
+        assert libdpo.check() == libdpo.OK
         outs.append((np64(tok), np64(dH), np64(dW)))
-    for o in outs[1:]:
+    for o in outs[1:4]:
         assert np.abs(outs[0][0] - o[0]).max() <= 1e-4
         assert rel_frob(outs[0][1], o[1]) <= 1e-3
         assert rel_frob(outs[0][2], o[2]) <= 1e-3
+    for o in outs[4:]:
+        for a, b in zip(outs[0], o):
+            assert np.array_equal(a, b)
 
 
 @pytest.mark.parametrize("R,L,d,V,seed", [
@@ -178,3 +185,31 @@ def test_maximum_sizes(R, L, d, V, seed):
     w = WL.make_custom(R=R, L=L, d=d, V=V, dtype="bf16", seed=seed, prompt_range=(1, 1),
                        min_completion=1)
     _fwd_bwd_check(w)
+
+
+@pytest.mark.parametrize("R,L,d,V,seed", [
+    (4, 600, 512, 5000, 111),      # 10 output tiles: dH split into K parts
+    (2, 900, 256, 70001, 112),     # long vocabulary, few tiles: one split launch, ragged K
+])
+def test_split_k_dh_against_the_oracle(R, L, d, V, seed):
+    """Shapes whose dH GEMM has too few output tiles to fill the GPU run it as K parts
+    of one launch (the workspace holds their fp32 partial sums); the parts are added in
+    a fixed order, so dH equals the oracle's within tolerance and repeats bit for bit."""
+    import torch
+    w = WL.make_custom(R=R, L=L, d=d, V=V, dtype="bf16", seed=seed, prompt_range=(1, L // 3),
+                       full_rows=1)
+    dw = DeviceWorkload(w)
+    _, bwd, _ = libdpo.workspace_size(dw.batch())
+    nc = w.n_scored
+    assert bwd >= nc * ((V + 7) // 8 * 8 * 2 + d * 4)      # dz rows + at least one part
+    _, _, lse = dw.forward(dw.W, want_grad=True)
+    coef = torch.from_numpy(np.random.default_rng(seed).normal(0, 0.05, R).astype(np.float32)).cuda()
+    dH1, dW1 = dw.backward(lse, coef)
+    dH2, dW2 = dw.backward(lse, coef)
+    assert libdpo.check() == libdpo.OK
+    assert torch.equal(dH1, dH2) and torch.equal(dW1, dW2)
+    Hd = WL.widen(w.H, "bf16")
+    oH, oW = O.backward(Hd, WL.widen(w.W, "bf16"), w.tokens, w.prompt_len, w.completion_len,
+                        coef.double().cpu().numpy())
+    assert rel_frob(np64(dH1), oH) <= TOL_GRAD
+    assert rel_frob(np64(dW1), oW) <= TOL_GRAD
