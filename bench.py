@@ -448,9 +448,13 @@ def run_ours(args):
     launches_per_step = (fwd_launches if fwd_only else 2 * fwd_launches + 1 + bwd_launches)
 
     if args.profile_step:
-        # a profiler's run: the given number of plain steps, nothing timed or printed
+        # a profiler's run: the given number of plain steps, nothing timed or printed (a
+        # forward-only run also makes one dpo_logits_mean call: it needs only H, W and the
+        # forward workspace)
         for _ in range(args.profile_step):
             step()
+        if args.forward_only:
+            libdpo.logits_mean(bp, w.layout, torch.empty(2, device=dev), ws, stream=sp)
         st = libdpo.check(sp)
         if ws_n > 1:
             dist.destroy_process_group()
@@ -702,8 +706,8 @@ def main(argv=None):
     ap.add_argument("--profile-step", type=int, default=0,
                     help="run this many untimed steps and exit (a profiler's command)")
     ap.add_argument("--forward-only", action="store_true",
-                    help="with --profile-step: the policy forward alone (weights, H and the "
-                         "forward workspace on the device, nothing else)")
+                    help="with --profile-step: the policy forward alone, then one logits-mean "
+                         "call (weights, H and the forward workspace on the device, nothing else)")
     raw = sys.argv[1:] if argv is None else list(argv)
     args = ap.parse_args(raw)
     if args.warmup < 3 and args.impl == "ours":
