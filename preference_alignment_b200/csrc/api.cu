@@ -137,11 +137,17 @@ struct Plan {
 // another SM count the choice is only less well tuned).
 constexpr int kPlanPairs = 74;
 constexpr int kMaxDhParts = 16;
+// A unit's epilogue (a 256 x 256 fp32 tile written out) takes about as long as this many
+// K blocks of MMAs; it overlaps the next unit's main loop, so a unit costs at least this.
+// It is also the shortest K part the split uses.
+constexpr int kEpilogueKb = 8;
 
 // Estimated duration of a launch of `units` work units of `kb` K blocks each, in units
 // of one K block on every pair: whole rounds of kPlanPairs units.
 double rounds_x_k(long long units, long long kb) {
-  return static_cast<double>((units + kPlanPairs - 1) / kPlanPairs) * static_cast<double>(kb);
+  const long long per_unit = kb > kEpilogueKb ? kb : kEpilogueKb;
+  return static_cast<double>((units + kPlanPairs - 1) / kPlanPairs) *
+         static_cast<double>(per_unit);
 }
 
 // dH = dz . W has few output tiles (token tiles x column tiles of d), so one launch can
@@ -169,6 +175,7 @@ void plan_dh_split(Plan* p) {
   for (int q = 2; q <= kMaxDhParts; ++q) {
     long long kbp = (kb + q - 1) / q;
     if (kbp > max_kbp) continue;
+    if (kbp < kEpilogueKb) break;
     const int parts = static_cast<int>((kb + kbp - 1) / kbp);
     const double est = rounds_x_k(tiles * parts, kbp) * (1.0 + 0.02 * (parts - 1));
     if (est < best * 0.97) {

@@ -83,6 +83,7 @@ def _run(name):
     res["n_rows"] = len(g_seq)
     if not backward:
         _CACHE[name] = res
+        print(f"\n{name}: " + ", ".join(f"{k} {v}" for k, v in res.items() if k not in ("w",)))
         return res
 
     res["lse_err"] = float(np.abs(np64(lse)[:w.n_scored] - op["lse"]).max())
@@ -126,6 +127,7 @@ def _run(name):
     del gH, oH, H64
     gc.collect()
     _CACHE[name] = res
+    print(f"\n{name}: " + ", ".join(f"{k} {v}" for k, v in res.items() if k not in ("w",)))
     return res
 
 
