@@ -501,10 +501,14 @@ def run_ours(args):
     # Every step uploads its inputs (H, tokens) from pinned host memory and reads its
     # results (loss and metrics) back. As a training loop would, the upload of step
     # i + 1 runs on a copy stream into the other of two input buffers while step i
-    # computes; the step waits for its own upload with an event.
+    # computes (the step waits for its own upload with an event), and the host reads
+    # step i's results once step i + 1 is queued behind it, so the GPU never idles
+    # while the host waits for a result.
     H_host = torch.from_numpy(np.ascontiguousarray(w.H).view(np.int16)).view(torch.bfloat16).pin_memory()
     tok_host = torch.from_numpy(w.tokens).pin_memory()
-    res_host = torch.empty(max(2 + 3 * B, w.R), dtype=torch.float32).pin_memory()
+    res_host = torch.empty(2, max(2 + 3 * B, w.R), dtype=torch.float32).pin_memory()
+    res_ready = [torch.cuda.Event() for _ in range(2)]
+    host_read = []
     e2e_steps = max(3, min(args.steps, 20))
     copy_stream = torch.cuda.Stream(dev)
     H_buf = [H, torch.empty_like(H)]
@@ -552,8 +556,13 @@ def run_ours(args):
             else:
                 res_dev = torch.cat([outs["loss"], outs["accuracy"], outs["margins"], outs["cr"],
                                      outs["rr"]])
-            res_host[:res_dev.numel()].copy_(res_dev, non_blocking=True)
-            stream.synchronize()                             # the host reads the step's result
+            res_host[i % 2, :res_dev.numel()].copy_(res_dev, non_blocking=True)
+            res_ready[i % 2].record(stream)
+            if i > 0:                                        # the host reads step i - 1
+                res_ready[(i - 1) % 2].synchronize()
+                host_read.append(float(res_host[(i - 1) % 2, 0]))
+        res_ready[(e2e_steps - 1) % 2].synchronize()         # and the last step
+        host_read.append(float(res_host[(e2e_steps - 1) % 2, 0]))
         e1.record(stream)
         torch.cuda.synchronize(dev)
         e2e_reps.append(e0.elapsed_time(e1))
@@ -688,9 +697,10 @@ def main(argv=None):
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(WL.CONFIGS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-cublas-reference", action="store_true")
-    ap.add_argument("--gemm-variant", type=int, default=0, choices=range(512),
+    ap.add_argument("--gemm-variant", type=int, default=0, choices=range(1024),
                     help="mask, per GEMM (forward, dz, dH, dW) bit k: single-CTA kernel, "
-                         "bit 4 + k: static tile schedule; bit 8: dH without split-K")
+                         "bit 4 + k: static tile schedule; bit 8: dH without split-K; "
+                         "bit 9: split-K dH for a long vocabulary too")
     ap.add_argument("--cpu-tokens-per-row", type=int, default=64,
                     help="oracle sample (CPU baseline and reference arm): completion tokens "
                          "per row of one pair")

@@ -166,7 +166,8 @@ void plan_dh_split(Plan* p) {
   p->dh_parts = 1;
   if (p->dtype != DPO_BF16 || tiles == 0 || ((gemm_variant() >> 8) & 1)) return;
   const double seq = rounds_x_k(tiles, kb);     // one launch or sequential chunks alike
-  if (p->V >= kDhChunkFrom &&
+  const bool force_split = (gemm_variant() >> 9) & 1;
+  if (p->V >= kDhChunkFrom && !force_split &&
       static_cast<double>(tiles) / ((tiles + kPlanPairs - 1) / kPlanPairs * kPlanPairs) >= 0.9)
     return;
   // the split with the fewest estimated K-block rounds, each extra part charged 2 %
@@ -178,7 +179,7 @@ void plan_dh_split(Plan* p) {
     if (kbp < kEpilogueKb) break;
     const int parts = static_cast<int>((kb + kbp - 1) / kbp);
     const double est = rounds_x_k(tiles * parts, kbp) * (1.0 + 0.02 * (parts - 1));
-    if (est < best * 0.97) {
+    if (est < best * 0.97 || (force_split && p->dh_parts == 1 && kbp * kBK <= kDhVocabChunk)) {
       best = est;
       p->dh_kb_part = static_cast<int>(kbp);
       p->dh_parts = parts;
@@ -766,7 +767,7 @@ dpo_status dpo_selftest_wait_timeout(uint32_t budget_ms, void* stream) {
 }
 
 int32_t dpo_set_gemm_variant(int32_t variant) {
-  if (variant < 0 || variant > 511) return -1;
+  if (variant < 0 || variant > 1023) return -1;
   return g_gemm_variant.exchange(variant);
 }
 

@@ -448,28 +448,39 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 
   if (warp == 0 && lane == 0) {
     // ---------------------------------------------------------------- TMA producer
-    // (the leader's also claims the pair's tiles and publishes them in the ring)
+    // The leader's producer also claims the pair's tiles and publishes them in the ring,
+    // one tile ahead: the claim of tile i + 1 is issued when tile i's loads start and
+    // published when they have all been issued, so the atomic's round trip overlaps the
+    // loads instead of stalling them at every tile boundary.
     const uint32_t full_leader = mapa_shared(full0, 0);
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
+    // Leader: wait (bounded) for slot i to be free, then write `tile` into both CTAs'
+    // copies of it and release-arrive on both CTAs' `full` barrier.
+    auto publish = [&](int i, int tile) -> bool {
+      const int slot = i % kSchedSlots;
+      const uint32_t ph = static_cast<uint32_t>(i / kSchedSlots) & 1u;
+      if (!mbar_wait(sempty0 + 8 * slot, ph ^ 1u, ctl, abort_flag)) return false;
+      for (uint32_t r = 0; r < 2; ++r) {
+        st_shared_cluster_u32(mapa_shared(ring.tile0 + 4 * slot, r), static_cast<uint32_t>(tile));
+        mbar_arrive_cluster(mapa_shared(sfull0 + 8 * slot, r));
+      }
+      return true;
+    };
+    int claimed = -1;                       // leader: the tile published in slot i
+    if (dyn && leader) {
+      claimed = atomicAdd(g.counter, 1);
+      if (claimed >= n_tiles_total) claimed = -1;
+      ok = publish(0, claimed);
+    }
     for (int i = 0; ok; ++i) {
       int tile = pair + i * n_pairs;
+      int next = -1;
       if (dyn) {
         if (leader) {
-          const int slot = i % kSchedSlots;
-          const uint32_t ph = static_cast<uint32_t>(i / kSchedSlots) & 1u;
-          if (!mbar_wait(sempty0 + 8 * slot, ph ^ 1u, ctl, abort_flag)) {
-            ok = false;
-            break;
-          }
-          tile = atomicAdd(g.counter, 1);
-          if (tile >= n_tiles_total) tile = -1;
-          for (uint32_t r = 0; r < 2; ++r) {
-            st_shared_cluster_u32(mapa_shared(ring.tile0 + 4 * slot, r),
-                                  static_cast<uint32_t>(tile));
-            mbar_arrive_cluster(mapa_shared(sfull0 + 8 * slot, r));
-          }
+          tile = claimed;
+          if (tile >= 0) next = atomicAdd(g.counter, 1);   // the result is used after the loads
         } else if (!ring.take(i, tile, ctl, abort_flag)) {
           ok = false;
           break;
@@ -507,6 +518,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           stage = 0;
           phase ^= 1;
         }
+      }
+      if (ok && dyn && leader) {
+        claimed = next < n_tiles_total ? next : -1;
+        ok = publish(i + 1, claimed);
       }
     }
     if (!ok) {
