@@ -39,8 +39,36 @@ WORKLOAD = "llama8b"
 CONFIG_TEXT = ("Llama-3.1-8B head shape: 4 pairs -> 8 rows, seq 2048, prompt U{256..1024}, "
                "completion to >=95% fill, d=4096, V=128256, bf16; policy fwd+bwd, reference fwd")
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-DH_VOCAB_CHUNK = 16384   # vocabulary columns per dH GEMM launch in the library's backward
-                         # (vocabularies of at least 4 chunks; shorter ones: one launch)
+
+
+def dh_launches(Nc, d, V, pairs=74):
+    """Kernel launches of the library's dH = dz.W for Nc positions (its plan, restated for
+    the launch count): sequential launches of 16,384 vocabulary columns for a vocabulary
+    of at least 65,536 whose launches fill >= 90 % of their rounds of 74 CTA pairs, else
+    one launch, split over the vocabulary into K parts (plus one reduce kernel) when the
+    parts fill the rounds better by the plan's estimate."""
+    kb = -(-V // 64)
+    tiles = -(-Nc // 256) * -(-d // 256)
+    if tiles == 0:
+        return 0
+
+    def est(units, k):
+        return -(-units // pairs) * max(k, 8)
+
+    if V >= 65536 and tiles / (-(-tiles // pairs) * pairs) >= 0.9:
+        return -(-V // 16384)
+    best, parts = est(tiles, kb), 1
+    for q in range(2, 17):
+        kbp = -(-kb // q)
+        if kbp > (1 << 20) // 64:
+            continue
+        if kbp < 8:
+            break
+        n = -(-kb // kbp)
+        e = est(tiles * n, kbp) * (1.0 + 0.02 * (n - 1))
+        if e < best * 0.97:
+            best, parts = e, n
+    return 2 if parts > 1 else (-(-V // 16384) if V >= 65536 else 1)
 
 
 # ------------------------------------------------------------------ helpers
@@ -436,15 +464,14 @@ def run_ours(args):
 
     # launches of our kernels per step: upload + prep + GEMM + combine + rowsum per forward,
     # one loss kernel; the backward (one token chunk: the workspace holds all Nc rows of
-    # dz) runs upload + prep + the dz GEMM + one dH GEMM per DH_VOCAB_CHUNK vocabulary
-    # columns + the dW GEMM
+    # dz) runs upload + prep + the dz GEMM + the dH launches (dh_launches) + the dW GEMM
     uploads = math.ceil(w.R / 1024)
     fwd_launches = uploads + 4
-    dh_launches = math.ceil(w.V / DH_VOCAB_CHUNK) if w.V >= 4 * DH_VOCAB_CHUNK else 1
+    n_dh = dh_launches(Nc, w.d, w.V)
     if ws_n > 1:   # dz, then dW by blocks of vocabulary rows, then dH
-        bwd_launches = uploads + 2 + len(DP.vocab_buckets(w.V, args.dw_buckets)) + dh_launches
+        bwd_launches = uploads + 2 + len(DP.vocab_buckets(w.V, args.dw_buckets)) + n_dh
     else:
-        bwd_launches = uploads + 3 + dh_launches
+        bwd_launches = uploads + 3 + n_dh
     launches_per_step = (fwd_launches if fwd_only else 2 * fwd_launches + 1 + bwd_launches)
 
     if args.profile_step:

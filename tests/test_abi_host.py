@@ -254,3 +254,27 @@ def test_shard_calls_reject_missing_outputs_and_workspace(lib):
         with pytest.raises(libdpo.DpoError) as e:
             libdpo.shard_combine(b, total, n, FAKE, FAKE, seq, None, None, FAKE, ws_bytes=1 << 30)
         assert e.value.status == libdpo.ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("R,L,d,V", [(16, 512, 2048, 32000), (8, 2048, 4096, 128256),
+                                     (4, 4096, 2048, 151936), (4, 300, 128, 700),
+                                     (2, 900, 256, 70001), (2, 8, 8, 1 << 24)])
+def test_dh_split_plan_matches_the_bench_launch_count(lib, R, L, d, V):
+    """The backward workspace holds split-K partial sums exactly when the library splits
+    dH over the vocabulary (compared with the diagnostic bit that turns the split off),
+    and bench.py's launch count restates the same plan."""
+    import bench
+    P = np.full(R, 1, np.int32)
+    C = np.full(R, L - 1, np.int32)
+    b = _batch(R=R, L=L, d=d, V=V, P=P, C=C)
+    _, bw_split, _ = libdpo.workspace_size(b)
+    old = libdpo.set_gemm_variant(256)
+    try:
+        _, bw_plain, _ = libdpo.workspace_size(b)
+    finally:
+        libdpo.set_gemm_variant(old)
+    nc = int(C.sum())
+    split = bw_split > bw_plain
+    assert (bench.dh_launches(nc, d, V) == 2) == split    # one split launch + its reduce
+    if split:                                             # >= one part's fp32 partial sums
+        assert bw_split - bw_plain >= nc * d * 4
