@@ -213,3 +213,25 @@ def test_split_k_dh_against_the_oracle(R, L, d, V, seed):
                         coef.double().cpu().numpy())
     assert rel_frob(np64(dH1), oH) <= TOL_GRAD
     assert rel_frob(np64(dW1), oW) <= TOL_GRAD
+
+
+def test_split_k_dh_in_a_chunked_backward():
+    """A workspace smaller than the whole batch's runs the backward in token chunks; with
+    dH split over K each chunk's partial sums sit after its dz rows. The result equals the
+    one-chunk backward within rounding (the dW chunks add in a different order)."""
+    import torch
+    w = WL.make_custom(R=4, L=600, d=512, V=5000, dtype="bf16", seed=113, prompt_range=(1, 200),
+                       full_rows=1)
+    dw = DeviceWorkload(w)
+    b = dw.batch()
+    _, full, mn = libdpo.workspace_size(b)
+    row = (full - mn) // max(1, w.n_scored - 128)          # bytes per position (dz + parts)
+    small = mn + 2 * 128 * row                             # 384 positions per chunk
+    assert row > ((w.V + 7) // 8 * 8) * 2 and small < full
+    _, _, lse = dw.forward(dw.W, want_grad=True)
+    coef = torch.from_numpy(np.random.default_rng(113).normal(0, 0.05, w.R).astype(np.float32)).cuda()
+    dH1, dW1 = dw.backward(lse, coef)
+    dH2, dW2 = dw.backward(lse, coef, ws_bytes=small)
+    assert libdpo.check() == libdpo.OK
+    assert rel_frob(np64(dH2), np64(dH1)) < 1e-6
+    assert rel_frob(np64(dW2), np64(dW1)) < 1e-5
