@@ -235,3 +235,32 @@ def test_split_k_dh_in_a_chunked_backward():
     assert libdpo.check() == libdpo.OK
     assert rel_frob(np64(dH2), np64(dH1)) < 1e-6
     assert rel_frob(np64(dW2), np64(dW1)) < 1e-5
+
+
+def test_workspace_contents_do_not_matter():
+    """The GEMMs' tile claim counter and every table live in the workspace; each call
+    writes what it reads (the counter is zeroed before each launch), so a workspace full
+    of garbage gives the same bits as a fresh one."""
+    import torch
+    w = WL.make_custom(R=6, L=300, d=256, V=3000, dtype="bf16", seed=114, prompt_range=(1, 100),
+                       full_rows=2)
+    dw = DeviceWorkload(w)
+    b = dw.batch()
+    fwd, bwd, _ = libdpo.workspace_size(b)
+    n = max(fwd, bwd)
+    coef = torch.linspace(-0.1, 0.2, w.R, device="cuda")
+    outs = []
+    for fill in (0x00, 0x7F, 0xFF):
+        ws = torch.full((n,), fill, dtype=torch.uint8, device="cuda")
+        seq = torch.empty(w.R, device="cuda")
+        lse = torch.empty(w.n_scored, device="cuda")
+        libdpo.seq_logprobs(b, True, seq, None, lse, ws)
+        dH = torch.empty(w.R, w.L, w.d, device="cuda")
+        dW = torch.empty(w.V, w.d, device="cuda")
+        ws.fill_(fill)
+        libdpo.backward(b, lse, coef, dH, dW, False, ws)
+        assert libdpo.check() == libdpo.OK
+        outs.append((seq, lse, dH, dW))
+    for o in outs[1:]:
+        for a, c in zip(outs[0], o):
+            assert torch.equal(a, c)
