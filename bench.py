@@ -4,8 +4,10 @@ One step = policy dpo_seq_logprobs(want_grad=1) + reference dpo_seq_logprobs
 + dpo_loss + dpo_backward, on the Llama-3.1-8B head shape (8 rows = 4
 chosen/rejected pairs, L = 2048, d = 4096, V = 128,256, bf16), synthetic seeded
 inputs. Under torchrun each rank runs its own pairs (data parallel, weak
-scaling) with the same weights; the step ends with an NCCL all-reduce of dW and
-of the loss, the exchange a data-parallel optimiser step needs.
+scaling) with the same weights: the loss call gets the whole batch's pair count
+(each rank's loss and coefficients are its share), and the backward forms dW by
+blocks of vocabulary rows, each block's NCCL all-reduce running while the next
+block is formed, then dH; one small all-reduce sums the loss shares.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -98,11 +100,14 @@ def _free_port():
 
 def launch_ranks(argv, n):
     """Re-run this script as n local ranks under torch.distributed.run (one process per
-    GPU); returns the launcher's exit status. NCCL's init log stays on (INFO) so a
-    scaling record shows the communicator's ranks, unless NCCL_DEBUG is already set."""
+    GPU); returns the launcher's exit status. NCCL's init log stays on (INFO, to stderr,
+    so stdout keeps only rank 0's JSON line) and shows the communicator's ranks, unless
+    NCCL_DEBUG is already set."""
     env = dict(os.environ)
-    env.setdefault("NCCL_DEBUG", "INFO")
-    env.setdefault("NCCL_DEBUG_SUBSYS", "INIT")
+    if "NCCL_DEBUG" not in env:
+        env["NCCL_DEBUG"] = "INFO"
+        env.setdefault("NCCL_DEBUG_SUBSYS", "INIT")
+        env.setdefault("NCCL_DEBUG_FILE", "/dev/stderr")
     cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
            "--master-addr=127.0.0.1", f"--master-port={_free_port()}",
            os.path.abspath(__file__), *argv]
@@ -366,10 +371,22 @@ def run_ours(args):
     ws_n, rank, local = dist_env()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    if ws_n > 1:
+    # the data-parallel step (exact shares, dW exchanged by blocks while the next block is
+    # formed) runs whenever there are several ranks; --dp-path runs it on one rank too (a
+    # one-rank NCCL group), which measures what its structure costs the GPU's compute
+    exch = ws_n > 1 or args.dp_path
+    if exch:
         import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=dev)
+        # NCCL's own messages (its version line, any debug log) go to stderr, so stdout
+        # holds only rank 0's JSON line
+        os.environ.setdefault("NCCL_DEBUG_FILE", "/dev/stderr")
+        if ws_n == 1:
+            store = dist.TCPStore("127.0.0.1", _free_port(), 1, True)
+            dist.init_process_group("nccl", store=store, rank=0, world_size=1,
+                                    timeout=datetime.timedelta(seconds=120), device_id=dev)
+        else:
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=dev)
     libdpo.load()
     libdpo.set_gemm_variant(args.gemm_variant)
 
@@ -417,7 +434,7 @@ def run_ours(args):
     # loss call gets the whole batch's pair count, so its loss, accuracy and row
     # coefficients are its share; one all-reduce sums the shares, the bucketed backward
     # sums dW.
-    pairs_total = DP.global_counts(B, 0, device=dev)[0] if ws_n > 1 else 0
+    pairs_total = DP.global_counts(B, 0, device=dev)[0] if exch else 0
     shares = torch.empty(2, device=dev)
     outs["loss"], outs["accuracy"] = shares[0:1], shares[1:2]
 
@@ -449,7 +466,7 @@ def run_ours(args):
                        pairs_total=pairs_total, stream=sp)
         if timed is not None:
             ev[3].record(stream)
-        if ws_n > 1:
+        if exch:
             works = DP.backward_exchange(bp, lse, outs["coef"], dH, dW, ws,
                                          n_buckets=args.dw_buckets,
                                          max_sms=max(2, sms - args.comm_sms))
@@ -468,7 +485,7 @@ def run_ours(args):
     uploads = math.ceil(w.R / 1024)
     fwd_launches = uploads + 4
     n_dh = dh_launches(Nc, w.d, w.V)
-    if ws_n > 1:   # dz, then dW by blocks of vocabulary rows, then dH
+    if exch:       # dz, then dW by blocks of vocabulary rows, then dH
         bwd_launches = uploads + 2 + len(DP.vocab_buckets(w.V, args.dw_buckets)) + n_dh
     else:
         bwd_launches = uploads + 3 + n_dh
@@ -483,7 +500,7 @@ def run_ours(args):
         if args.forward_only:
             libdpo.logits_mean(bp, w.layout, torch.empty(2, device=dev), ws, stream=sp)
         st = libdpo.check(sp)
-        if ws_n > 1:
+        if exch:
             dist.destroy_process_group()
         return 0 if st == libdpo.OK else 1
 
@@ -669,6 +686,8 @@ def run_ours(args):
                        "pairs_per_gpu": B, "seq_len": w.L, "d": w.d, "V": w.V,
                        "scored_tokens_per_gpu": Nc, "global_batch_pairs": B * ws_n,
                        "parallelism": f"dp{ws_n}",
+                       "dw_exchange": (f"{args.dw_buckets} blocks of vocabulary rows, "
+                                       f"{args.comm_sms} SMs left to NCCL") if exch else None,
                        "l2": "inputs larger than L2 (W and W_ref are 1.05 GB each; no flush)"},
             "pct_of_peak": {"algorithmic": alg_flop * args.steps / (ms / 1e3) / 1e12 / sustained,
                             "executed": exe_flop * args.steps / (ms / 1e3) / 1e12 / sustained,
@@ -709,8 +728,9 @@ def run_ours(args):
             "logits_fp32_bytes_avoided": 4 * Nc * w.V,
         }
         print(json.dumps(line), flush=True)
-    if ws_n > 1:
-        dist.barrier()
+    if exch:
+        if ws_n > 1:
+            dist.barrier()
         dist.destroy_process_group()
     return 0
 
@@ -737,6 +757,9 @@ def main(argv=None):
                     help="data parallel: blocks of dW rows whose all-reduce overlaps the next")
     ap.add_argument("--comm-sms", type=int, default=16,
                     help="data parallel: SMs the backward GEMMs leave free for NCCL")
+    ap.add_argument("--dp-path", action="store_true",
+                    help="run the data-parallel step (bucketed dW exchange) on a single rank "
+                         "too, to measure what its structure costs")
     ap.add_argument("--pairs", type=int, default=0,
                     help="keep only the workload's first P pairs (a smaller case, e.g. for a "
                          "profiler); 0 = all")
