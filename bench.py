@@ -423,7 +423,13 @@ def run_ours(args):
     ref = torch.empty(w.R, device=dev)
     lse = torch.empty(Nc, device=dev)
     dH = torch.empty(w.R, w.L, w.d, device=dev) if not fwd_only else None
-    dW = torch.empty(w.V, w.d, device=dev) if not fwd_only else None
+    scatter = None
+    if exch and args.dw_exchange == "scatter" and not fwd_only:
+        # dW reduce-scattered inside the dW GEMM: each rank ends with its block of rows
+        scatter = DP.FusedReduceScatter(w.V, w.d, device=dev)
+        dW = torch.empty(len(scatter.rows), w.d, device=dev)
+    else:
+        dW = torch.empty(w.V, w.d, device=dev) if not fwd_only else None
     outs = {k: torch.empty(n, device=dev) for k, n in
             [("loss", 1), ("accuracy", 1), ("margins", B), ("cr", B), ("rr", B), ("w", B),
              ("coef", 2 * B)]}
@@ -466,7 +472,11 @@ def run_ours(args):
                        pairs_total=pairs_total, stream=sp)
         if timed is not None:
             ev[3].record(stream)
-        if exch:
+        if scatter is not None:
+            scatter.backward(bp, lse, outs["coef"], dH, dW, ws,
+                             max_sms=max(2, sms - args.comm_sms))
+            DP.allreduce_shares(shares)
+        elif exch:
             works = DP.backward_exchange(bp, lse, outs["coef"], dH, dW, ws,
                                          n_buckets=args.dw_buckets,
                                          max_sms=max(2, sms - args.comm_sms))
@@ -485,7 +495,9 @@ def run_ours(args):
     uploads = math.ceil(w.R / 1024)
     fwd_launches = uploads + 4
     n_dh = dh_launches(Nc, w.d, w.V)
-    if exch:       # dz, then dW by blocks of vocabulary rows, then dH
+    if scatter is not None:   # dz, the scatter dW GEMM, dH, the owner's sum of its slots
+        bwd_launches = uploads + 2 + 1 + n_dh + 1
+    elif exch:     # dz, then dW by blocks of vocabulary rows, then dH
         bwd_launches = uploads + 2 + len(DP.vocab_buckets(w.V, args.dw_buckets)) + n_dh
     else:
         bwd_launches = uploads + 3 + n_dh
@@ -501,6 +513,9 @@ def run_ours(args):
             libdpo.logits_mean(bp, w.layout, torch.empty(2, device=dev), ws, stream=sp)
         st = libdpo.check(sp)
         if exch:
+            if scatter is not None:
+                dist.barrier()
+                scatter.close()
             dist.destroy_process_group()
         return 0 if st == libdpo.OK else 1
 
@@ -686,8 +701,12 @@ def run_ours(args):
                        "pairs_per_gpu": B, "seq_len": w.L, "d": w.d, "V": w.V,
                        "scored_tokens_per_gpu": Nc, "global_batch_pairs": B * ws_n,
                        "parallelism": f"dp{ws_n}",
-                       "dw_exchange": (f"{args.dw_buckets} blocks of vocabulary rows, "
-                                       f"{args.comm_sms} SMs left to NCCL") if exch else None,
+                       "dw_exchange": (None if not exch else
+                                       f"reduce-scatter fused into the dW GEMM (CUDA IPC "
+                                       f"receive buffers), {args.comm_sms} SMs left free"
+                                       if scatter is not None else
+                                       f"all-reduce of {args.dw_buckets} blocks of vocabulary "
+                                       f"rows, {args.comm_sms} SMs left to NCCL"),
                        "l2": "inputs larger than L2 (W and W_ref are 1.05 GB each; no flush)"},
             "pct_of_peak": {"algorithmic": alg_flop * args.steps / (ms / 1e3) / 1e12 / sustained,
                             "executed": exe_flop * args.steps / (ms / 1e3) / 1e12 / sustained,
@@ -729,6 +748,10 @@ def run_ours(args):
         }
         print(json.dumps(line), flush=True)
     if exch:
+        if scatter is not None:
+            torch.cuda.synchronize(dev)
+            dist.barrier()
+            scatter.close()
         if ws_n > 1:
             dist.barrier()
         dist.destroy_process_group()
@@ -757,6 +780,9 @@ def main(argv=None):
                     help="data parallel: blocks of dW rows whose all-reduce overlaps the next")
     ap.add_argument("--comm-sms", type=int, default=16,
                     help="data parallel: SMs the backward GEMMs leave free for NCCL")
+    ap.add_argument("--dw-exchange", choices=["allreduce", "scatter"], default="allreduce",
+                    help="data parallel: NCCL all-reduce of dW blocks overlapped with the "
+                         "backward, or the reduce-scatter fused into the dW GEMM")
     ap.add_argument("--dp-path", action="store_true",
                     help="run the data-parallel step (bucketed dW exchange) on a single rank "
                          "too, to measure what its structure costs")

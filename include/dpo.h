@@ -214,6 +214,54 @@ dpo_status dpo_backward_dw(const dpo_batch* batch, int32_t v_begin, int32_t v_en
 dpo_status dpo_backward_dh(const dpo_batch* batch, float* dH, int32_t max_sms, void* ws,
                            size_t ws_bytes, void* stream);
 
+/* ---- Data-parallel exchange fused into the dW GEMM ---------------------------
+ * With the pairs split across ranks (each rank its own pairs, the same W), dW is the
+ * sum over ranks of each rank's dz_r^T . Hp_r. As a reduce-scatter fused into the dW
+ * GEMM: rank q owns a block of W's rows; every rank forms its whole contribution and
+ * its GEMM epilogue stores each finished row straight into the owner's receive buffer,
+ * in this rank's slot (another process's buffer, mapped with dpo_ipc_import: peer
+ * memory over NVLink when the ranks run on different GPUs), so the transfer proceeds
+ * tile by tile while the GEMM runs. After a barrier on every rank (an all-reduce of one
+ * number on the same stream is one), each owner adds its slots in rank order
+ * (dpo_dw_reduce_slots) and holds its block of the summed dW, as a sharded optimiser
+ * needs ("Run Distributed Full-Model DPO with PyTorch FSDP", Step 1). Deterministic:
+ * the sum is taken in rank order. */
+#define DPO_MAX_SCATTER_RANKS 8
+typedef struct {
+  int32_t n_ranks;          /* 1 .. DPO_MAX_SCATTER_RANKS                                 */
+  int32_t rank;             /* this rank, 0 .. n_ranks - 1                                */
+  int32_t rows_per_rank;    /* rank q < n_ranks - 1 owns W rows [q * rows_per_rank, +rows_per_rank);
+                               the last rank owns the rest (at least one row)             */
+  float* recv[DPO_MAX_SCATTER_RANKS];  /* recv[q]: rank q's receive buffer [n_ranks, rows_q,
+                               d] fp32, 16-byte aligned, as this process addresses it     */
+} dpo_dw_scatter;
+
+/* This rank's contribution to dW (the dz that a preceding dpo_backward(dW = NULL) left in
+ * ws, times the batch's packed H), each row stored into its owner's buffer at slot
+ * `rank` (recv[q] + (rank * rows_q + row - q * rows_per_rank) * d). bf16 batches only
+ * (DPO_ERR_UNSUPPORTED otherwise). The epilogue fences its stores at system scope before
+ * the kernel ends. max_sms and workspace errors as for dpo_backward_dw; a bad scatter
+ * description is DPO_ERR_INVALID_ARG. A batch with no scored position zeroes its slots. */
+dpo_status dpo_backward_dw_scatter(const dpo_batch* batch, const dpo_dw_scatter* scatter,
+                                   int32_t max_sms, void* ws, size_t ws_bytes, void* stream);
+
+/* The owner's side: dW_shard (+)= slot 0 + slot 1 + ... in slot order, over a receive
+ * buffer recv [n_slots, rows, d] fp32 (both 16-byte aligned; d a multiple of 8). Call it
+ * after every rank's dpo_backward_dw_scatter has completed (a barrier). */
+dpo_status dpo_dw_reduce_slots(const float* recv, int32_t n_slots, int32_t rows, int32_t d,
+                               float* dW_shard, int accumulate, void* stream);
+
+/* CUDA IPC of a device buffer between processes (the receive buffers above).
+ * dpo_ipc_export: the handle of the allocation that holds ptr (this process's device
+ * memory), and ptr's byte offset in it. dpo_ipc_import (in another process): map that
+ * allocation, peer access enabled; the buffer is at *base + offset. dpo_ipc_close: unmap. */
+typedef struct {
+  unsigned char bytes[64];
+} dpo_ipc_handle;
+dpo_status dpo_ipc_export(const void* ptr, dpo_ipc_handle* handle, size_t* offset);
+dpo_status dpo_ipc_import(const dpo_ipc_handle* handle, void** base);
+dpo_status dpo_ipc_close(void* base);
+
 /* ---- Vocabulary-parallel head ----------------------------------------------
  * W split by vocabulary rows across ranks, every rank holding the same batch (the
  * vocabulary-parallel alternative to data parallelism for a head too large to

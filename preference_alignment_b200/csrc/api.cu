@@ -681,6 +681,59 @@ dpo_status dpo_backward_dw(const dpo_batch* batch, int32_t v_begin, int32_t v_en
                 accumulate_dW ? 1 : 0, sm_budget(di, max_sms), make_ctl(di), st);
 }
 
+static_assert(DPO_MAX_SCATTER_RANKS == dpo::kMaxScatterRanks, "one limit of scatter ranks");
+
+dpo_status dpo_backward_dw_scatter(const dpo_batch* batch, const dpo_dw_scatter* sc_arg,
+                                   int32_t max_sms, void* ws, size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_range("dpo_backward_dw_scatter");
+  Plan p;
+  dpo_status s = make_plan(batch, &p);
+  if (s != DPO_OK) return s;
+  if (p.dtype != DPO_BF16) return DPO_ERR_UNSUPPORTED;
+  if (sc_arg == nullptr) return DPO_ERR_INVALID_ARG;
+  const dpo_dw_scatter& x = *sc_arg;
+  if (x.n_ranks < 1 || x.n_ranks > kMaxScatterRanks || x.rank < 0 || x.rank >= x.n_ranks ||
+      x.rows_per_rank < 1 || static_cast<long long>(x.rows_per_rank) * (x.n_ranks - 1) >= p.V)
+    return DPO_ERR_INVALID_ARG;
+  for (int q = 0; q < x.n_ranks; ++q)
+    if (x.recv[q] == nullptr || !aligned16(x.recv[q])) return DPO_ERR_INVALID_ARG;
+  if ((s = dz_resident(p, ws, ws_bytes, max_sms)) != DPO_OK) return s;
+  DevInfo di;
+  if ((s = device_info(&di)) != DPO_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (p.Nc == 0) {                      // no scored position: this rank's slots are zero
+    for (int q = 0; q < x.n_ranks; ++q) {
+      const long long first = static_cast<long long>(q) * x.rows_per_rank;
+      const long long rows_q = q == x.n_ranks - 1 ? p.V - first : x.rows_per_rank;
+      if (cudaMemsetAsync(x.recv[q] + static_cast<size_t>(x.rank) * rows_q * p.d, 0,
+                          sizeof(float) * static_cast<size_t>(rows_q) * p.d, st) != cudaSuccess)
+        return DPO_ERR_CUDA;
+    }
+    return DPO_OK;
+  }
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  const uint16_t* G = reinterpret_cast<const uint16_t*>(w + p.off_G);
+  const uint16_t* Hp = reinterpret_cast<const uint16_t*>(w + p.off_hp);
+  CUtensorMap mGmn, mHmn;
+  if (!make_map(&mGmn, G, p.V, p.Nc, 2ull * p.ldG, kBoxMN, kBK) ||
+      !make_map(&mHmn, Hp, p.d, p.Nc, 2ull * p.d, kBoxMN, kBK))
+    return DPO_ERR_CUDA;
+  const Sched sc = sched_of(p, ws);
+  return cuda_status(launch_bwd_dw_scatter(mGmn, mHmn, p.Nc, p.V, p.d, x.recv, x.n_ranks, x.rank,
+                                           x.rows_per_rank, sm_budget(di, max_sms), sc.sync,
+                                           make_ctl(di), st));
+}
+
+dpo_status dpo_dw_reduce_slots(const float* recv, int32_t n_slots, int32_t rows, int32_t d,
+                               float* dW_shard, int accumulate, void* stream) {
+  NvtxRange nvtx_range("dpo_dw_reduce_slots");
+  if (recv == nullptr || dW_shard == nullptr || !aligned16(recv) || !aligned16(dW_shard) ||
+      n_slots < 1 || n_slots > kMaxScatterRanks || rows < 0 || d < 8 || d % 8 != 0)
+    return DPO_ERR_INVALID_ARG;
+  return cuda_status(launch_dw_reduce_slots(recv, n_slots, rows, d, dW_shard, accumulate ? 1 : 0,
+                                            static_cast<cudaStream_t>(stream)));
+}
+
 dpo_status dpo_backward_dh(const dpo_batch* batch, float* dH, int32_t max_sms, void* ws,
                            size_t ws_bytes, void* stream) {
   NvtxRange nvtx_range("dpo_backward_dh");

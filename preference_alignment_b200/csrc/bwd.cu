@@ -31,6 +31,7 @@ constexpr float kLog2eB = 1.4426950408889634f;
 // from it two chunks earlier has finished reading it.
 struct EpiGrad {
   static constexpr bool kStaging = true;   // stores through TMA staging buffers
+  static constexpr bool kSystemFence = false;
   struct Params {
     const int* y;
     const float* lse;
@@ -104,6 +105,7 @@ struct EpiGrad {
 // to the rows in part order.
 struct EpiRows {
   static constexpr bool kStaging = false;   // stores go straight to global memory
+  static constexpr bool kSystemFence = false;
   struct Params {
     const int* dst;        // packed position -> flat row r * L + t
     float* out;            // dH [R * L, d]
@@ -183,6 +185,7 @@ __global__ void __launch_bounds__(256) k_dh_reduce(float* __restrict__ dH,
 // ------------------------------------------------------------------ dW epilogue
 struct EpiDW {
   static constexpr bool kStaging = false;   // stores go straight to global memory
+  static constexpr bool kSystemFence = false;
   struct Params {
     float* out;            // dW [V, d]
     int V, d, accumulate;
@@ -222,6 +225,109 @@ struct EpiDW {
 
   __device__ __forceinline__ void end(const Params&) {}
 };
+
+// ------------------------------------------------------------------ dW scatter epilogue
+// The data-parallel exchange fused into the dW GEMM, as a reduce-scatter: the vocabulary
+// rows are owned by ranks in blocks (rank q owns rows [q * rows_per_rank, ...), the last
+// rank the rest), and each finished row of this rank's contribution dz_r^T . Hp_r is
+// stored straight into its owner's receive buffer, in this rank's slot. The owner's
+// buffer is another process's memory mapped into this one (peer memory over NVLink when
+// that process runs on another GPU), so the transfer happens tile by tile while the GEMM
+// runs; the epilogue threads fence at system scope before the kernel ends, so a barrier
+// after the kernel (on every rank) makes every rank's rows visible to their owners,
+// who then add the slots in rank order (k_dw_reduce_slots).
+struct EpiDWScatter {
+  static constexpr bool kStaging = false;   // plain stores to (peer) global memory
+  static constexpr bool kSystemFence = true;
+  struct Params {
+    float* recv[kMaxScatterRanks];   // recv[q]: rank q's buffer [n_ranks, rows_q, d]
+    int V, d, n_ranks, rank, rows_per_rank;
+  };
+  float* o;
+  int nbase;
+  bool valid;
+
+  __device__ __forceinline__ void begin(const Params& p, int m_row, int nt, int,
+                                        const EpiCtx&) {
+    const int v = m_row;
+    valid = v < p.V;
+    nbase = nt * kBN;
+    o = nullptr;
+    if (!valid) return;
+    const int q = min(v / p.rows_per_rank, p.n_ranks - 1);
+    const int first = q * p.rows_per_rank;
+    const int rows_q = q == p.n_ranks - 1 ? p.V - first : p.rows_per_rank;
+    o = p.recv[q] + (static_cast<long long>(p.rank) * rows_q + (v - first)) * p.d;
+  }
+
+  __device__ __forceinline__ void chunk(const Params& p, int c, const uint32_t (&v)[32]) {
+    if (!valid) return;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int col = nbase + c * 32 + q * 4;
+      if (col < p.d)
+        *reinterpret_cast<float4*>(o + col) =
+            make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
+                        __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
+    }
+  }
+
+  __device__ __forceinline__ void end(const Params&) {}
+};
+
+// out[row] (+)= slot 0[row] + slot 1[row] + ... (slots in rank order, fp32, one thread per
+// 4 columns): the owner's side of the reduce-scatter, over its [n_slots, rows, d] buffer.
+__global__ void __launch_bounds__(256) k_dw_reduce_slots(const float* __restrict__ recv,
+                                                         int n_slots, long long rows_x_d4,
+                                                         float* __restrict__ out,
+                                                         int accumulate) {
+  const long long q = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (q >= rows_x_d4) return;
+  const float4* src = reinterpret_cast<const float4*>(recv) + q;
+  float4 a = __ldg(src);
+  for (int s = 1; s < n_slots; ++s) {
+    const float4 b = __ldg(src + s * rows_x_d4);
+    a.x += b.x;
+    a.y += b.y;
+    a.z += b.z;
+    a.w += b.w;
+  }
+  float4* o = reinterpret_cast<float4*>(out) + q;
+  if (accumulate) {
+    const float4 old = *o;
+    a.x += old.x;
+    a.y += old.y;
+    a.z += old.z;
+    a.w += old.w;
+  }
+  *o = a;
+}
+
+cudaError_t launch_bwd_dw_scatter(const CUtensorMap& mapA, const CUtensorMap& mapB, int Mc, int V,
+                                  int d, float* const* recv, int n_ranks, int rank,
+                                  int rows_per_rank, int grid, int* sync, const DevCtl& ctl,
+                                  cudaStream_t st) {
+  if (n_ranks < 1 || n_ranks > kMaxScatterRanks) return cudaErrorInvalidValue;
+  EpiDWScatter::Params p{};
+  for (int q = 0; q < n_ranks; ++q) p.recv[q] = recv[q];
+  p.V = V;
+  p.d = d;
+  p.n_ranks = n_ranks;
+  p.rank = rank;
+  p.rows_per_rank = rows_per_rank;
+  return launch_gemm<true, true, EpiDWScatter>(mapA, mapB, mapA, V, d, Mc,
+                                               DPO_GROUP_DW > 0 ? 3 : 1, p, grid, ctl, st,
+                                               kGemmDW, DPO_GROUP_DW, sync);
+}
+
+cudaError_t launch_dw_reduce_slots(const float* recv, int n_slots, int rows, int d, float* out,
+                                   int accumulate, cudaStream_t st) {
+  const long long n4 = static_cast<long long>(rows) * (d / 4);
+  if (n4 == 0) return cudaSuccess;
+  k_dw_reduce_slots<<<static_cast<unsigned>((n4 + 255) / 256), 256, 0, st>>>(recv, n_slots, n4,
+                                                                            out, accumulate);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_bwd_grad(const CUtensorMap& mapA, const CUtensorMap& mapB,
                             const CUtensorMap& mapG, int Mc, int V, int d, int tok0, const int* y,

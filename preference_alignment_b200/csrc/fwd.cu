@@ -83,6 +83,7 @@ cudaError_t launch_prep(const uint16_t* H, const int* tokens, const Sched& s, in
 // One thread = one packed position (accumulator row), 256 vocab columns per tile.
 struct EpiLSE {
   static constexpr bool kStaging = false;   // stores go straight to global memory
+  static constexpr bool kSystemFence = false;
   struct Params {
     const int* y;
     float2* part;

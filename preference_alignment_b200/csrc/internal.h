@@ -109,6 +109,19 @@ cudaError_t launch_bwd_dw(const CUtensorMap& mapA, const CUtensorMap& mapB, int 
                           float* dW, int accumulate, int grid, int* sync, const DevCtl& ctl,
                           cudaStream_t st);
 
+// Data-parallel reduce-scatter fused into the dW GEMM (at most kMaxScatterRanks ranks):
+// row v of this rank's dW contribution goes to recv[q] (rank q's buffer [n_ranks, rows_q,
+// d], q = the owner of v) at slot `rank`; rank q owns rows [q * rows_per_rank, ...), the
+// last rank the rest.
+constexpr int kMaxScatterRanks = 8;   // DPO_MAX_SCATTER_RANKS
+cudaError_t launch_bwd_dw_scatter(const CUtensorMap& mapA, const CUtensorMap& mapB, int Mc, int V,
+                                  int d, float* const* recv, int n_ranks, int rank,
+                                  int rows_per_rank, int grid, int* sync, const DevCtl& ctl,
+                                  cudaStream_t st);
+// out (+)= sum over the n_slots slots of recv ([n_slots, rows, d]), slots in order.
+cudaError_t launch_dw_reduce_slots(const float* recv, int n_slots, int rows, int d, float* out,
+                                   int accumulate, cudaStream_t st);
+
 // Loss kernel (fp64 inside). pairs_total / nll_tokens_total: the whole data-parallel
 // batch's pair count and chosen-token count (0: this call's own).
 cudaError_t launch_loss(int B, int layout, const float* pol, const float* ref, double beta,

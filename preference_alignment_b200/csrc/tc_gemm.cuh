@@ -302,8 +302,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
 
   // Bulk stores an epilogue issued must finish before the CTA (and its shared
-  // memory) goes away; warps that issued none return at once.
+  // memory) goes away; warps that issued none return at once. An epilogue whose stores
+  // go to another process's memory (Epi::kSystemFence) fences them at system scope.
   if (warp >= 2 && lane == 0) bulk_wait_group<0>();
+  if constexpr (Epi::kSystemFence) {
+    if (warp >= 2) __threadfence_system();
+  }
 
   // ---------------------------------------------------------------- teardown
   __syncthreads();
@@ -457,11 +461,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     uint32_t phase = 0;
     bool ok = true;
     // Leader: wait (bounded) for slot i to be free, then write `tile` into both CTAs'
-    // copies of it and release-arrive on both CTAs' `full` barrier.
+    // copies of it and release-arrive on both CTAs' `full` barrier. The wait acquires at
+    // cluster scope: readers in the other CTA release the slot with a release-arrive.
     auto publish = [&](int i, int tile) -> bool {
       const int slot = i % kSchedSlots;
       const uint32_t ph = static_cast<uint32_t>(i / kSchedSlots) & 1u;
-      if (!mbar_wait(sempty0 + 8 * slot, ph ^ 1u, ctl, abort_flag)) return false;
+      if (!mbar_wait_cluster(sempty0 + 8 * slot, ph ^ 1u, ctl, abort_flag)) return false;
       for (uint32_t r = 0; r < 2; ++r) {
         st_shared_cluster_u32(mapa_shared(ring.tile0 + 4 * slot, r), static_cast<uint32_t>(tile));
         mbar_arrive_cluster(mapa_shared(sfull0 + 8 * slot, r));
@@ -641,8 +646,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   }
 
   // Bulk stores an epilogue issued must finish before the CTA (and its shared
-  // memory) goes away; warps that issued none return at once.
+  // memory) goes away; warps that issued none return at once. An epilogue whose stores
+  // go to another process's memory (Epi::kSystemFence) fences them at system scope.
   if (warp >= 2 && lane == 0) bulk_wait_group<0>();
+  if constexpr (Epi::kSystemFence) {
+    if (warp >= 2) __threadfence_system();
+  }
 
   // ---------------------------------------------------------------- teardown
   __syncthreads();

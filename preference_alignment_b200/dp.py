@@ -90,3 +90,97 @@ def backward_exchange(batch, lse_state, row_coef, dH, dW, ws, n_buckets=8, max_s
     if dH is not None:
         libdpo.backward_dh(batch, dH, ws, max_sms=max_sms)
     return works
+
+
+# ------------------------------------------------------------------ fused reduce-scatter
+def scatter_rows_per_rank(V: int, n_ranks: int, align: int = ROW_ALIGN) -> int:
+    """Rows of W each rank but the last owns in the fused reduce-scatter: whole `align`-row
+    tiles, as even as possible, the last rank owning the rest (at least one row)."""
+    if V < n_ranks or n_ranks < 1:
+        raise ValueError("need at least one vocabulary row per rank")
+    tiles = (V + align - 1) // align
+    per = -(-tiles // n_ranks) * align
+    while per > align and per * (n_ranks - 1) >= V:
+        per -= align
+    if per * (n_ranks - 1) >= V:          # fewer tiles than ranks: rows, not tiles
+        per = V // n_ranks
+    return per
+
+
+def scatter_rows(V: int, n_ranks: int, q: int, per: int) -> range:
+    """The rows of W rank q owns."""
+    return range(q * per, V if q == n_ranks - 1 else (q + 1) * per)
+
+
+class FusedReduceScatter:
+    """The data-parallel dW exchange fused into the dW GEMM, as a reduce-scatter.
+
+    Rank q owns rows scatter_rows(V, n, q, per) of dW and holds a receive buffer
+    [n, rows_q, d] fp32 with one slot per rank. The buffers are shared between the
+    processes with CUDA IPC (each rank maps every other rank's buffer), so each rank's
+    dW GEMM stores every finished row of its contribution straight into the owner's
+    slot (peer memory over NVLink between GPUs) while the GEMM runs; after a barrier
+    each owner adds its slots in rank order (the same bits on every run) and holds its
+    rows of the summed dW, as a sharded optimiser ("Run Distributed Full-Model DPO
+    with PyTorch FSDP", Step 1) needs.
+
+    barrier: called with no arguments where every rank must have finished the work
+    enqueued so far. The default is an all-reduce of one number on the current stream
+    (NCCL: the host does not wait); for a process group whose collectives are not
+    ordered on the stream (gloo), pass one that synchronizes the device first.
+    """
+
+    def __init__(self, V: int, d: int, group=None, device=None, barrier=None):
+        import torch
+        import torch.distributed as dist
+        from preference_alignment_b200 import libdpo
+        self.group = group
+        self.rank = dist.get_rank(group)
+        self.n = dist.get_world_size(group)
+        if self.n > libdpo.MAX_SCATTER_RANKS:
+            raise ValueError(f"at most {libdpo.MAX_SCATTER_RANKS} ranks")
+        self.V, self.d = V, d
+        self.per = scatter_rows_per_rank(V, self.n)
+        self.rows = scatter_rows(V, self.n, self.rank, self.per)
+        dev = device if device is not None else torch.device("cuda", torch.cuda.current_device())
+        self.recv = torch.empty(self.n, len(self.rows), d, dtype=torch.float32, device=dev)
+        handle, offset = libdpo.ipc_export(self.recv)
+        shared = [None] * self.n
+        dist.all_gather_object(shared, (handle, offset), group=group)
+        self.mapped = []
+        self.ptrs = []
+        for q, (h, off) in enumerate(shared):
+            if q == self.rank:
+                self.ptrs.append(self.recv.data_ptr())
+            else:
+                base = libdpo.ipc_import(h)
+                self.mapped.append(base)
+                self.ptrs.append(base + off)
+        self._flag = torch.zeros(1, device=dev)
+        self.barrier = barrier if barrier is not None else self._stream_barrier
+
+    def _stream_barrier(self):
+        import torch.distributed as dist
+        dist.all_reduce(self._flag, group=self.group)
+
+    def backward(self, batch, lse_state, row_coef, dH, dW_shard, ws, max_sms=0,
+                 accumulate=False):
+        """dz (dpo_backward with dW = NULL), this rank's dW rows scattered to their owners,
+        dH, then the barrier and the sum of this rank's slots into dW_shard ([rows_q, d];
+        added to when accumulate), then a second barrier so that no rank's next scatter
+        reaches a buffer whose slots are still being summed."""
+        from preference_alignment_b200 import libdpo
+        libdpo.backward(batch, lse_state, row_coef, None, None, False, ws)
+        libdpo.backward_dw_scatter(batch, self.n, self.rank, self.per, self.ptrs, ws,
+                                   max_sms=max_sms)
+        if dH is not None:
+            libdpo.backward_dh(batch, dH, ws, max_sms=max_sms)
+        self.barrier()
+        libdpo.dw_reduce_slots(self.recv, self.n, len(self.rows), self.d, dW_shard, accumulate)
+        self.barrier()
+
+    def close(self):
+        from preference_alignment_b200 import libdpo
+        for base in self.mapped:
+            libdpo.ipc_close(base)
+        self.mapped = []

@@ -237,6 +237,81 @@ def backward_dh(batch: BatchArgs, dH, ws, ws_bytes=None, max_sms: int = 0, strea
               _stream(stream)), "dpo_backward_dh")
 
 
+MAX_SCATTER_RANKS = 8
+
+
+class DwScatter(ctypes.Structure):
+    _fields_ = [("n_ranks", ctypes.c_int32), ("rank", ctypes.c_int32),
+                ("rows_per_rank", ctypes.c_int32),
+                ("recv", ctypes.c_void_p * MAX_SCATTER_RANKS)]
+
+
+def backward_dw_scatter(batch: BatchArgs, n_ranks: int, rank: int, rows_per_rank: int, recv, ws,
+                        ws_bytes=None, max_sms: int = 0, stream=None):
+    """dpo_backward_dw_scatter: this rank's dW contribution, each row stored into its owner's
+    receive buffer (recv: one device address or tensor per rank, as this process maps it)."""
+    lib = load()
+    fn = lib.dpo_backward_dw_scatter
+    vp = ctypes.c_void_p
+    fn.argtypes = [ctypes.POINTER(Batch), ctypes.POINTER(DwScatter), ctypes.c_int32, vp,
+                   ctypes.c_size_t, vp]
+    fn.restype = ctypes.c_int
+    ptrs = [_ptr(r) for r in recv]
+    if len(ptrs) != n_ranks or n_ranks > MAX_SCATTER_RANKS:
+        raise ValueError("recv needs one buffer per rank (at most 8 ranks)")
+    x = DwScatter(int(n_ranks), int(rank), int(rows_per_rank),
+                  (ctypes.c_void_p * MAX_SCATTER_RANKS)(*(ptrs + [None] * (MAX_SCATTER_RANKS - n_ranks))))
+    _check(fn(ctypes.byref(batch.c), ctypes.byref(x), int(max_sms), _ptr(ws), _nbytes(ws, ws_bytes),
+              _stream(stream)), "dpo_backward_dw_scatter")
+
+
+def dw_reduce_slots(recv, n_slots: int, rows: int, d: int, dW_shard, accumulate: bool = False,
+                    stream=None):
+    """dpo_dw_reduce_slots: dW_shard (+)= the sum of recv's n_slots slots, in slot order."""
+    lib = load()
+    fn = lib.dpo_dw_reduce_slots
+    vp = ctypes.c_void_p
+    fn.argtypes = [vp, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, vp, ctypes.c_int, vp]
+    fn.restype = ctypes.c_int
+    _check(fn(_ptr(recv), int(n_slots), int(rows), int(d), _ptr(dW_shard), 1 if accumulate else 0,
+              _stream(stream)), "dpo_dw_reduce_slots")
+
+
+class IpcHandle(ctypes.Structure):
+    _fields_ = [("bytes", ctypes.c_ubyte * 64)]
+
+
+def ipc_export(ptr):
+    """dpo_ipc_export: (64-byte handle as bytes, byte offset) of the allocation holding ptr."""
+    lib = load()
+    fn = lib.dpo_ipc_export
+    fn.argtypes = [ctypes.c_void_p, ctypes.POINTER(IpcHandle), ctypes.POINTER(ctypes.c_size_t)]
+    fn.restype = ctypes.c_int
+    h, off = IpcHandle(), ctypes.c_size_t()
+    _check(fn(_ptr(ptr), ctypes.byref(h), ctypes.byref(off)), "dpo_ipc_export")
+    return bytes(h.bytes), off.value
+
+
+def ipc_import(handle: bytes) -> int:
+    """dpo_ipc_import: map another process's exported allocation; returns its base address."""
+    lib = load()
+    fn = lib.dpo_ipc_import
+    fn.argtypes = [ctypes.POINTER(IpcHandle), ctypes.POINTER(ctypes.c_void_p)]
+    fn.restype = ctypes.c_int
+    h = IpcHandle((ctypes.c_ubyte * 64)(*handle))
+    base = ctypes.c_void_p()
+    _check(fn(ctypes.byref(h), ctypes.byref(base)), "dpo_ipc_import")
+    return base.value
+
+
+def ipc_close(base: int):
+    lib = load()
+    fn = lib.dpo_ipc_close
+    fn.argtypes = [ctypes.c_void_p]
+    fn.restype = ctypes.c_int
+    _check(fn(base), "dpo_ipc_close")
+
+
 class VocabShard(ctypes.Structure):
     _fields_ = [("offset", ctypes.c_int32), ("total", ctypes.c_int32)]
 

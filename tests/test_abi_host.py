@@ -278,3 +278,53 @@ def test_dh_split_plan_matches_the_bench_launch_count(lib, R, L, d, V):
     assert (bench.dh_launches(nc, d, V) == 2) == split    # one split launch + its reduce
     if split:                                             # >= one part's fp32 partial sums
         assert bw_split - bw_plain >= nc * d * 4
+
+
+@pytest.mark.parametrize("n_ranks,rank,per,recv,code", [
+    (0, 0, 50, FAKE, libdpo.ERR_INVALID_ARG),        # no ranks
+    (9, 0, 10, FAKE, libdpo.ERR_INVALID_ARG),        # beyond DPO_MAX_SCATTER_RANKS
+    (2, 2, 50, FAKE, libdpo.ERR_INVALID_ARG),        # rank out of range
+    (2, -1, 50, FAKE, libdpo.ERR_INVALID_ARG),
+    (3, 0, 50, FAKE, libdpo.ERR_INVALID_ARG),        # the last rank would own no row (V 100)
+    (2, 0, 0, FAKE, libdpo.ERR_INVALID_ARG),         # no rows per rank
+    (2, 0, 50, FAKE + 4, libdpo.ERR_INVALID_ARG),    # a misaligned receive buffer
+    (2, 0, 50, 0, libdpo.ERR_INVALID_ARG),           # a missing receive buffer
+])
+def test_backward_dw_scatter_rejects(lib, n_ranks, rank, per, recv, code):
+    """The library's own checks, through the raw call (all 8 buffer slots filled)."""
+    import ctypes
+    b = _batch()
+    x = libdpo.DwScatter(n_ranks, rank, per)
+    for i in range(libdpo.MAX_SCATTER_RANKS):
+        x.recv[i] = recv
+    st = lib.dpo_backward_dw_scatter(ctypes.byref(b.c), ctypes.byref(x), 0, FAKE, 1 << 30, None)
+    assert st == code
+
+
+def test_backward_dw_scatter_refuses_fp32_and_small_workspaces(lib):
+    with pytest.raises(libdpo.DpoError) as e:
+        libdpo.backward_dw_scatter(_batch(dtype="f32"), 1, 0, 100, [FAKE], FAKE, ws_bytes=1 << 30)
+    assert e.value.status == libdpo.ERR_UNSUPPORTED
+    b = _batch(L=128, C=[100, 100, 100, 100])
+    _, bw, mn = libdpo.workspace_size(b)
+    with pytest.raises(libdpo.DpoError) as e:
+        libdpo.backward_dw_scatter(b, 1, 0, 100, [FAKE], FAKE, ws_bytes=mn)
+    assert e.value.status == libdpo.ERR_WORKSPACE
+
+
+@pytest.mark.parametrize("kw", [dict(n_slots=0), dict(n_slots=9), dict(d=12), dict(rows=-1),
+                                dict(recv=FAKE + 4), dict(out=None)])
+def test_dw_reduce_slots_rejects(lib, kw):
+    a = dict(recv=FAKE, n_slots=2, rows=10, d=64, out=FAKE)
+    a.update(kw)
+    with pytest.raises(libdpo.DpoError) as e:
+        libdpo.dw_reduce_slots(a["recv"], a["n_slots"], a["rows"], a["d"], a["out"])
+    assert e.value.status == libdpo.ERR_INVALID_ARG
+
+
+def test_ipc_calls_fail_cleanly_without_device_memory(lib):
+    with pytest.raises(libdpo.DpoError):
+        libdpo.ipc_export(FAKE)                      # not device memory of this process
+    with pytest.raises(libdpo.DpoError) as e:
+        libdpo.ipc_close(0)
+    assert e.value.status == libdpo.ERR_INVALID_ARG

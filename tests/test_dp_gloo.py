@@ -155,3 +155,18 @@ def test_rank_batch_without_weights_matches_full_draw():
     assert light.W is None and light.W_ref is None
     for k in ("prompt_len", "completion_len", "tokens", "H"):
         assert np.array_equal(getattr(full, k), getattr(light, k))
+
+
+def test_scatter_rows_partition_the_vocabulary():
+    for V, n in [(128256, 8), (1000, 3), (300, 4), (256, 2), (5, 4), (151936, 8), (70001, 2),
+                 (1, 1)]:
+        per = DP.scatter_rows_per_rank(V, n)
+        rows = [DP.scatter_rows(V, n, q, per) for q in range(n)]
+        assert rows[0].start == 0 and rows[-1].stop == V
+        assert all(a.stop == b.start for a, b in zip(rows, rows[1:]))
+        assert all(len(r) > 0 for r in rows)
+        assert all(len(r) == per for r in rows[:-1])
+        if V >= 256 * n:
+            assert per % 256 == 0                    # whole tiles of the dW GEMM
+    with pytest.raises(ValueError):
+        DP.scatter_rows_per_rank(3, 4)
