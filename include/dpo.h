@@ -253,8 +253,11 @@ dpo_status dpo_dw_reduce_slots(const float* recv, int32_t n_slots, int32_t rows,
 
 /* CUDA IPC of a device buffer between processes (the receive buffers above).
  * dpo_ipc_export: the handle of the allocation that holds ptr (this process's device
- * memory), and ptr's byte offset in it. dpo_ipc_import (in another process): map that
- * allocation, peer access enabled; the buffer is at *base + offset. dpo_ipc_close: unmap. */
+ * memory from cudaMalloc, as PyTorch's default allocator makes it; memory mapped through
+ * the virtual-memory API, such as PyTorch's expandable segments, is refused with
+ * DPO_ERR_CUDA), and ptr's byte offset in it; DPO_ERR_INVALID_ARG when ptr is not device
+ * memory of this process. dpo_ipc_import (in another process): map that allocation, peer
+ * access enabled; the buffer is at *base + offset. dpo_ipc_close: unmap. */
 typedef struct {
   unsigned char bytes[64];
 } dpo_ipc_handle;
