@@ -149,13 +149,17 @@ class FusedReduceScatter:
         dist.all_gather_object(shared, (handle, offset), group=group)
         self.mapped = []
         self.ptrs = []
-        for q, (h, off) in enumerate(shared):
-            if q == self.rank:
-                self.ptrs.append(self.recv.data_ptr())
-            else:
-                base = libdpo.ipc_import(h)
-                self.mapped.append(base)
-                self.ptrs.append(base + off)
+        try:
+            for q, (h, off) in enumerate(shared):
+                if q == self.rank:
+                    self.ptrs.append(self.recv.data_ptr())
+                else:
+                    base = libdpo.ipc_import(h)
+                    self.mapped.append(base)
+                    self.ptrs.append(base + off)
+        except Exception:
+            self.close()                    # unmap what was mapped before the failure
+            raise
         self._flag = torch.zeros(1, device=dev)
         self.barrier = barrier if barrier is not None else self._stream_barrier
 
