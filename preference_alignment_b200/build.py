@@ -55,14 +55,21 @@ def build(force: bool = False, verbose: bool = False, extra=()) -> str:
     objs = []
     tmpdir = os.path.join(PKG, "_build")
     os.makedirs(tmpdir, exist_ok=True)
+    cmds = []
     for src in sources():
         obj = os.path.join(tmpdir, os.path.basename(src) + ".o")
         cmd = [nvcc, *ARCH, *FLAGS, *extra, "-I", INCLUDE, "-I", CSRC, "-c", src, "-o", obj]
         if verbose:
             cmd += ["-Xptxas", "-v"]
             print(" ".join(cmd), flush=True)
-        subprocess.run(cmd, check=True)
+        cmds.append(cmd)
         objs.append(obj)
+    # one nvcc per source file, as many at a time as the host has cores
+    from concurrent.futures import ThreadPoolExecutor
+    with ThreadPoolExecutor(max_workers=max(1, min(len(cmds), os.cpu_count() or 1))) as pool:
+        for r in list(pool.map(lambda c: subprocess.run(c), cmds)):
+            if r.returncode != 0:
+                raise subprocess.CalledProcessError(r.returncode, r.args)
     os.makedirs(os.path.dirname(LIB), exist_ok=True)
     tmp_lib = LIB + ".tmp"
     cmd = [nvcc, *ARCH, "-shared", "-o", tmp_lib, *objs, "-lcudart_static", "-ldl", "-lpthread", "-lrt"]
