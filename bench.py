@@ -45,10 +45,9 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 def dh_launches(Nc, d, V, pairs=74):
     """Kernel launches of the library's dH = dz.W for Nc positions (its plan, restated for
-    the launch count): sequential launches of 16,384 vocabulary columns for a vocabulary
-    of at least 65,536 whose launches fill >= 90 % of their rounds of 74 CTA pairs, else
-    one launch, split over the vocabulary into K parts (plus one reduce kernel) when the
-    parts fill the rounds better by the plan's estimate."""
+    the launch count): one launch over the vocabulary (in chunks of 2^20 columns beyond
+    that), or one launch split over the vocabulary into K parts plus one reduce kernel
+    when the parts fill the rounds of 74 CTA pairs better by the plan's estimate."""
     kb = -(-V // 64)
     tiles = -(-Nc // 256) * -(-d // 256)
     if tiles == 0:
@@ -57,8 +56,6 @@ def dh_launches(Nc, d, V, pairs=74):
     def est(units, k):
         return -(-units // pairs) * max(k, 8)
 
-    if V >= 65536 and tiles / (-(-tiles // pairs) * pairs) >= 0.9:
-        return -(-V // 16384)
     best, parts = est(tiles, kb), 1
     for q in range(2, 17):
         kbp = -(-kb // q)
@@ -70,7 +67,7 @@ def dh_launches(Nc, d, V, pairs=74):
         e = est(tiles * n, kbp) * (1.0 + 0.02 * (n - 1))
         if e < best * 0.97:
             best, parts = e, n
-    return 2 if parts > 1 else (-(-V // 16384) if V >= 65536 else 1)
+    return 2 if parts > 1 else -(-V // (1 << 20))
 
 
 # ------------------------------------------------------------------ helpers
@@ -767,10 +764,9 @@ def main(argv=None):
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(WL.CONFIGS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-cublas-reference", action="store_true")
-    ap.add_argument("--gemm-variant", type=int, default=0, choices=range(1024),
+    ap.add_argument("--gemm-variant", type=int, default=0, choices=range(512),
                     help="mask, per GEMM (forward, dz, dH, dW) bit k: single-CTA kernel, "
-                         "bit 4 + k: static tile schedule; bit 8: dH without split-K; "
-                         "bit 9: split-K dH for a long vocabulary too")
+                         "bit 4 + k: static tile schedule; bit 8: dH without split-K")
     ap.add_argument("--cpu-tokens-per-row", type=int, default=64,
                     help="oracle sample (CPU baseline and reference arm): completion tokens "
                          "per row of one pair")

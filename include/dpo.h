@@ -403,14 +403,11 @@ dpo_status dpo_selftest_wait_timeout(uint32_t budget_ms, void* stream);
  *              workspace (the tiles in flight stay one contiguous window of the
  *              raster); set: static round-robin (pair p takes tiles p, p + pairs, ...).
  *   bit 8      set: dH = dz.W is never split over the vocabulary (K) into parts of one
- *              launch (clear: split when that fills the GPU's waves better);
- *   bit 9      set: a long vocabulary whose dH launches already fill the GPU is split
- *              too (one launch in parts of at most 16,384 columns instead of sequential
- *              launches of 16,384 columns); bits 8 and 9 change the backward workspace
- *              size, so set them before sizing.
+ *              launch (clear: split when that fills the GPU's waves better); this bit
+ *              changes the backward workspace size, so set it before sizing.
  * Every choice gives the same results within rounding (bits 4-7 bit for bit: each tile
  * is computed the same way). Default 0. Returns the previous mask, or -1 for a value
- * outside 0..1023. A diagnostic for measurements; the default is the fastest measured. */
+ * outside 0..511. A diagnostic for measurements; the default is the fastest measured. */
 int32_t dpo_set_gemm_variant(int32_t variant);
 
 /* Static description of a status code. */

@@ -154,22 +154,15 @@ double rounds_x_k(long long units, long long kb) {
 // leave most of its last wave idle (e.g. 96 tiles on 74 pairs: 2 rounds for 1.3 waves of
 // work). Cutting the vocabulary (K) into parts that run as separate work units of one
 // launch fills the rounds; each part beyond the first costs an fp32 partial sum of the
-// rows (written, then added in part order by a small kernel). A long vocabulary that
-// already fills its rounds keeps sequential launches of kDhVocabChunk columns (measured
-// at the Llama-3.1-8B head: short K loops keep concurrent tiles close in K, so more
-// operand tiles come from L2).
+// rows (written, then added in part order by a small kernel).
 void plan_dh_split(Plan* p) {
   const long long kb = (p->V + kBK - 1) / kBK;
   const long long tiles = static_cast<long long>((p->Nc + 255) / 256) * ((p->d + kBN - 1) / kBN);
-  p->dh_chunk = p->V >= kDhChunkFrom ? kDhVocabChunk : kMaxAccumK;
+  p->dh_chunk = kMaxAccumK;                     // one launch unless the vocabulary exceeds it
   p->dh_kb_part = 0;
   p->dh_parts = 1;
   if (p->dtype != DPO_BF16 || tiles == 0 || ((gemm_variant() >> 8) & 1)) return;
-  const double seq = rounds_x_k(tiles, kb);     // one launch or sequential chunks alike
-  const bool force_split = (gemm_variant() >> 9) & 1;
-  if (p->V >= kDhChunkFrom && !force_split &&
-      static_cast<double>(tiles) / ((tiles + kPlanPairs - 1) / kPlanPairs * kPlanPairs) >= 0.9)
-    return;
+  const double seq = rounds_x_k(tiles, kb);
   // the split with the fewest estimated K-block rounds, each extra part charged 2 %
   const long long max_kbp = kMaxAccumK / kBK;   // K blocks one accumulation may take
   double best = seq;
@@ -179,7 +172,7 @@ void plan_dh_split(Plan* p) {
     if (kbp < kEpilogueKb) break;
     const int parts = static_cast<int>((kb + kbp - 1) / kbp);
     const double est = rounds_x_k(tiles * parts, kbp) * (1.0 + 0.02 * (parts - 1));
-    if (est < best * 0.97 || (force_split && p->dh_parts == 1 && kbp * kBK <= kDhVocabChunk)) {
+    if (est < best * 0.97) {
       best = est;
       p->dh_kb_part = static_cast<int>(kbp);
       p->dh_parts = parts;
@@ -373,9 +366,9 @@ float* dh_part_scratch(const Plan& p, uint8_t* w, int mc) {
 
 // dH rows of the packed positions [tok0, tok0 + mc) from the dz chunk in the workspace:
 // dH = dz . W, reduced over the vocabulary in one launch (split into K parts when that
-// fills the GPU's waves better, see plan_dh_split) or in sequential chunks of
-// kDhVocabChunk columns for a long vocabulary, the later chunks added to the rows by
-// the epilogue. No accumulation runs longer than kMaxAccumK products.
+// fills the GPU's waves better, see plan_dh_split); a vocabulary beyond kMaxAccumK
+// columns runs in chunks of that many, the later chunks added to the rows by the
+// epilogue. No accumulation runs longer than kMaxAccumK products.
 dpo_status run_dh(const Plan& p, const dpo_batch* batch, uint8_t* w, const Sched& sc, int tok0,
                   int mc, float* dH, int sms, const DevCtl& ctl, cudaStream_t st) {
   if (p.dtype != DPO_BF16) {
@@ -820,7 +813,7 @@ dpo_status dpo_selftest_wait_timeout(uint32_t budget_ms, void* stream) {
 }
 
 int32_t dpo_set_gemm_variant(int32_t variant) {
-  if (variant < 0 || variant > 1023) return -1;
+  if (variant < 0 || variant > 511) return -1;
   return g_gemm_variant.exchange(variant);
 }
 
