@@ -175,10 +175,17 @@ def dpo_loss(pol, ref, beta, layout="halves", grad_scale=1.0, completion_len=Non
     with nll_tokens_total = N_g the NLL divides by N_g; the outputs are then this
     part's share of the whole batch's values, and the shares of a partition of the
     batch add up to the values of the whole.
+
+    Reference-free objective (ref=None; "Run Distributed Full-Model DPO with PyTorch
+    FSDP", "Where to Go Next": it skips the frozen reference model; the formula is
+    not given there): the reference sums are read as 0, so the log-ratios are the
+    policy's own (normalised) sums, rewards beta * pi and margin beta * (pi_c - pi_r).
     """
     pol = [float(x) for x in pol]
-    ref = [float(x) for x in ref]
     R = len(pol)
+    ref = [0.0] * R if ref is None else [float(x) for x in ref]
+    if len(ref) != R:
+        raise ValueError("policy and reference sums differ in length")
     if R % 2:
         raise ValueError("odd number of rows")
     B = R // 2

@@ -373,6 +373,67 @@ def test_variant_row_coef_by_finite_differences(normalize, nll):
             assert out["row_coef"][r] == pytest.approx(fd, rel=1e-6, abs=1e-12)
 
 
+@pytest.mark.parametrize("normalize", [False, True])
+def test_reference_free_is_any_reference_that_ties_each_pair(normalize):
+    """The reference-free objective equals the referenced one whenever each pair's two
+    reference values (as the loss uses them) are equal, whatever that value: the
+    margins, losses, weights, accuracy and row coefficients agree, and the rewards
+    differ by beta times the tied value."""
+    rng = np.random.default_rng(36)
+    B = 6
+    C = rng.integers(1, 40, 2 * B)
+    pol = -rng.uniform(0.5, 4, 2 * B) * C
+    tie = rng.normal(0, 50, B)
+    for layout in ("halves", "adjacent"):
+        ref = np.empty(2 * B)
+        for i, (c, r) in enumerate(O.pair_rows(B, layout)):
+            # the value the loss sees is ref / C when normalising, ref otherwise
+            ref[c] = tie[i] * (C[c] if normalize else 1)
+            ref[r] = tie[i] * (C[r] if normalize else 1)
+        kw = dict(completion_len=C, normalize=normalize, nll_weight=0.3)
+        free = O.dpo_loss(pol, None, 0.1, layout, grad_scale=0.5, **kw)
+        tied = O.dpo_loss(pol, ref, 0.1, layout, grad_scale=0.5, **kw)
+        for k in ("margins", "losses", "weights", "row_coef"):
+            np.testing.assert_allclose(free[k], tied[k], rtol=1e-12, atol=1e-14)
+        for k in ("loss", "accuracy", "nll"):
+            assert free[k] == pytest.approx(tied[k], rel=1e-12, abs=1e-15)
+        np.testing.assert_allclose(free["chosen_rewards"], tied["chosen_rewards"] + 0.1 * tie,
+                                   rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(free["rejected_rewards"],
+                                   tied["rejected_rewards"] + 0.1 * tie, rtol=1e-12, atol=1e-12)
+
+
+def test_reference_free_on_the_worked_example_policy():
+    """The worked example's policy sums (-42.0 chosen, -47.5 rejected, beta 0.1) with no
+    reference: rewards are beta times the sums, the margin 0.55, one correct pair."""
+    out = O.dpo_loss([-42.0, -47.5], None, 0.1, "adjacent")
+    assert out["chosen_rewards"][0] == pytest.approx(-4.2, abs=1e-15)
+    assert out["rejected_rewards"][0] == pytest.approx(-4.75, abs=1e-15)
+    assert out["margins"][0] == pytest.approx(0.55, abs=1e-15)
+    assert out["accuracy"] == 1.0
+    # the referenced example's loss (0.576, margin 0.25) is larger: the margin grew
+    assert out["loss"] < O.dpo_loss([-42.0, -47.5], [-43.0, -46.0], 0.1, "adjacent")["loss"]
+
+
+@pytest.mark.parametrize("normalize,nll", [(False, 0.0), (True, 0.5)])
+def test_reference_free_row_coef_by_finite_differences(normalize, nll):
+    rng = np.random.default_rng(37)
+    B = 3
+    C = rng.integers(1, 30, 2 * B)
+    pol = -rng.uniform(0.05, 0.4, 2 * B) * C
+    kw = dict(completion_len=C, normalize=normalize, nll_weight=nll)
+    for layout in ("halves", "adjacent"):
+        out = O.dpo_loss(pol, None, 0.1, layout, grad_scale=0.5, **kw)
+        eps = 1e-5
+        for r in range(2 * B):
+            p1, p2 = pol.copy(), pol.copy()
+            p1[r] += eps
+            p2[r] -= eps
+            fd = 0.5 * (O.dpo_loss(p1, None, 0.1, layout, **kw)["loss"]
+                        - O.dpo_loss(p2, None, 0.1, layout, **kw)["loss"]) / (2 * eps)
+            assert out["row_coef"][r] == pytest.approx(fd, rel=1e-6, abs=1e-12)
+
+
 @pytest.mark.parametrize("normalize,nll", [(False, 0.0), (True, 0.0), (False, 0.6), (True, 0.4)])
 def test_data_parallel_shares_add_up_to_the_whole_batch(normalize, nll):
     """Shares of a partition of the pairs into unequal parts (1, 2 and 4 pairs), each
