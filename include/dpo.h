@@ -153,16 +153,24 @@ dpo_status dpo_loss(int32_t B, int32_t layout, const float* pol, const float* re
  * whole batch's values: summing them over the ranks (one all-reduce) gives the
  * single-process result on the whole batch, for unequal shards too ("Run
  * Distributed Full-Model DPO with PyTorch FSDP", Step 1: every rank holds part of
- * the global batch). Margins, rewards and weights are per pair and unchanged. */
+ * the global batch). Margins, rewards and weights are per pair and unchanged.
+ *   reference_free  1: the reference-free objective ("Run Distributed Full-Model DPO
+ *                   with PyTorch FSDP", "Where to Go Next": it skips the frozen
+ *                   reference model; the pages give no formula): the reference sums
+ *                   are read as 0, so rewards are beta * pi (normalised when asked)
+ *                   and the margin beta * (pi_c - pi_r); ref is not read and may be
+ *                   NULL. Composes with the options above. */
 typedef struct {
   int32_t normalize;
   float nll_weight;
   const int32_t* completion_len;
   int32_t pairs_total;      /* 0, or B_g >= B: the pairs of the whole data-parallel batch */
   int64_t nll_tokens_total; /* 0, or N_g >= 0: the whole batch's chosen completion tokens */
+  int32_t reference_free;   /* 0, or 1: no reference model (ref may be NULL) */
 } dpo_loss_options;
 
 /* dpo_loss with the variants above (opt may be NULL: then it equals dpo_loss).
+ * ref is required (DPO_ERR_INVALID_ARG when NULL) unless opt->reference_free is set.
  * row_coef stays d(grad_scale * loss)/d pol[row] and feeds dpo_backward as is.
  *   nll   device [1] or NULL: the NLL value (0 when nll_weight is 0) */
 dpo_status dpo_loss_ex(int32_t B, int32_t layout, const float* pol, const float* ref, float beta,

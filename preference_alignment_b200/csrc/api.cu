@@ -614,7 +614,10 @@ dpo_status dpo_loss_ex(int32_t B, int32_t layout, const float* pol, const float*
   NvtxRange nvtx_range("dpo_loss_ex");
   if (B < 1 || B > (1 << 28) || (layout != DPO_PAIRS_HALVES && layout != DPO_PAIRS_ADJACENT))
     return DPO_ERR_INVALID_ARG;
-  if (pol == nullptr || ref == nullptr || loss == nullptr) return DPO_ERR_INVALID_ARG;
+  const bool reference_free = opt != nullptr && opt->reference_free != 0;
+  if (reference_free) ref = nullptr;   // the kernel reads a NULL reference as zeros
+  if (pol == nullptr || (ref == nullptr && !reference_free) || loss == nullptr)
+    return DPO_ERR_INVALID_ARG;
   if (!(beta > 0.f) || !std::isfinite(beta) || !std::isfinite(grad_scale))
     return DPO_ERR_INVALID_ARG;
   int normalize = 0;
@@ -631,10 +634,12 @@ dpo_status dpo_loss_ex(int32_t B, int32_t layout, const float* pol, const float*
     if ((normalize || nll_weight > 0.f) && clen == nullptr) return DPO_ERR_INVALID_ARG;
     if (pairs_total != 0 && pairs_total < B) return DPO_ERR_INVALID_ARG;
     if (ntok_total < 0) return DPO_ERR_INVALID_ARG;
+    if (opt->reference_free != 0 && opt->reference_free != 1) return DPO_ERR_INVALID_ARG;
   }
   return cuda_status(launch_loss(B, layout, pol, ref, beta, grad_scale, normalize, nll_weight,
-                                 clen, pairs_total, ntok_total, loss, accuracy, margins, chosen_rewards, rejected_rewards,
-                                 weights, row_coef, nll, static_cast<cudaStream_t>(stream)));
+                                 clen, pairs_total, ntok_total, loss, accuracy, margins,
+                                 chosen_rewards, rejected_rewards, weights, row_coef, nll,
+                                 static_cast<cudaStream_t>(stream)));
 }
 
 dpo_status dpo_backward(const dpo_batch* batch, const float* lse_state, const float* row_coef,
@@ -832,6 +837,6 @@ const char* dpo_status_string(dpo_status s) {
   return "unknown status";
 }
 
-int32_t dpo_version(void) { return 200; }
+int32_t dpo_version(void) { return 300; }
 
 }  // extern "C"

@@ -14,6 +14,9 @@
 // nll_tokens_total = N_g the NLL term divides by the whole batch's chosen tokens, so
 // loss, accuracy, nll and row_coef are this rank's share of the global values: their
 // sum over ranks equals the single-process result on the whole batch.
+//
+// Reference-free objective ("Run Distributed Full-Model DPO with PyTorch FSDP",
+// "Where to Go Next"; no formula there): ref == NULL reads every reference sum as 0.
 #include <cmath>
 
 #include "internal.h"
@@ -52,8 +55,10 @@ __global__ void __launch_bounds__(256) k_dpo_loss(int B, int layout, const float
       sc = clen[c] > 0 ? 1.0 / clen[c] : 0.0;
       sr = clen[r] > 0 ? 1.0 / clen[r] : 0.0;
     }
-    const double rho_c = static_cast<double>(pol[c]) * sc - static_cast<double>(ref[c]) * sc;
-    const double rho_r = static_cast<double>(pol[r]) * sr - static_cast<double>(ref[r]) * sr;
+    const double ref_c = ref != nullptr ? static_cast<double>(ref[c]) : 0.0;
+    const double ref_r = ref != nullptr ? static_cast<double>(ref[r]) : 0.0;
+    const double rho_c = static_cast<double>(pol[c]) * sc - ref_c * sc;
+    const double rho_r = static_cast<double>(pol[r]) * sr - ref_r * sr;
     const double m = beta * (rho_c - rho_r);
     const double w = sigmoid_d(-m);
     lsum += softplus_d(-m);

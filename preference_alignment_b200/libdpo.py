@@ -179,16 +179,17 @@ def loss(B: int, layout, pol, ref, beta: float, grad_scale: float, loss_out, acc
 class LossOptions(ctypes.Structure):
     _fields_ = [("normalize", ctypes.c_int32), ("nll_weight", ctypes.c_float),
                 ("completion_len", ctypes.c_void_p), ("pairs_total", ctypes.c_int32),
-                ("nll_tokens_total", ctypes.c_int64)]
+                ("nll_tokens_total", ctypes.c_int64), ("reference_free", ctypes.c_int32)]
 
 
 def loss_ex(B: int, layout, pol, ref, beta: float, grad_scale: float, loss_out, accuracy=None,
             margins=None, chosen_rewards=None, rejected_rewards=None, weights=None, row_coef=None,
             nll=None, normalize=False, nll_weight=0.0, completion_len=None, pairs_total=0,
-            nll_tokens_total=0, stream=None):
+            nll_tokens_total=0, reference_free=False, stream=None):
     """dpo_loss_ex: length-normalised and/or SFT-NLL variants (completion_len: device int32 [2B]);
     pairs_total / nll_tokens_total > 0 make the outputs this rank's share of a data-parallel
-    batch of that many pairs / chosen tokens."""
+    batch of that many pairs / chosen tokens; reference_free reads the reference sums as 0
+    (ref is then not read and may be None)."""
     lib = load()
     fn = lib.dpo_loss_ex
     vp = ctypes.c_void_p
@@ -196,7 +197,7 @@ def loss_ex(B: int, layout, pol, ref, beta: float, grad_scale: float, loss_out, 
                    ctypes.POINTER(LossOptions), vp, vp, vp, vp, vp, vp, vp, vp, vp]
     fn.restype = ctypes.c_int
     opt = LossOptions(1 if normalize else 0, float(nll_weight), _ptr(completion_len),
-                      int(pairs_total), int(nll_tokens_total))
+                      int(pairs_total), int(nll_tokens_total), 1 if reference_free else 0)
     lay = LAYOUTS[layout] if isinstance(layout, str) else int(layout)
     _check(fn(int(B), lay, _ptr(pol), _ptr(ref), float(beta), float(grad_scale), ctypes.byref(opt),
               _ptr(loss_out), _ptr(accuracy), _ptr(margins), _ptr(chosen_rewards),

@@ -46,7 +46,7 @@ def test_status_strings_and_version(lib):
     for code in range(7):
         assert libdpo.status_string(code)
     assert libdpo.status_string(99) == "unknown status"
-    assert libdpo.version() == 200
+    assert libdpo.version() == 300
 
 
 FAKE = 0x10000  # never dereferenced: every call below fails its host checks first
@@ -201,6 +201,26 @@ def test_loss_ex_rejects_bad_options(lib, kw):
     with pytest.raises(libdpo.DpoError) as e:
         libdpo.loss_ex(2, "halves", FAKE, FAKE, 0.1, 1.0, FAKE, **kw)
     assert e.value.status == libdpo.ERR_INVALID_ARG
+
+
+def test_loss_needs_a_reference_unless_reference_free(lib):
+    with pytest.raises(libdpo.DpoError) as e:
+        libdpo.loss_ex(2, "halves", FAKE, None, 0.1, 1.0, FAKE)
+    assert e.value.status == libdpo.ERR_INVALID_ARG
+    with pytest.raises(libdpo.DpoError) as e:
+        libdpo.loss(2, "halves", FAKE, None, 0.1, 1.0, FAKE)
+    assert e.value.status == libdpo.ERR_INVALID_ARG
+
+
+def test_loss_ex_rejects_a_reference_free_flag_other_than_0_or_1(lib):
+    fn = lib.dpo_loss_ex
+    vp = ctypes.c_void_p
+    fn.argtypes = [ctypes.c_int32, ctypes.c_int32, vp, vp, ctypes.c_float, ctypes.c_float,
+                   ctypes.POINTER(libdpo.LossOptions), vp, vp, vp, vp, vp, vp, vp, vp, vp]
+    fn.restype = ctypes.c_int
+    opt = libdpo.LossOptions(0, 0.0, None, 0, 0, 2)
+    assert fn(2, 0, FAKE, None, 0.1, 1.0, ctypes.byref(opt), FAKE, None, None, None, None, None,
+              None, None, None) == libdpo.ERR_INVALID_ARG
 
 
 @pytest.mark.parametrize("kw,layout,means,ws,code", [

@@ -13,7 +13,7 @@ pytestmark = pytest.mark.gpu
 
 
 def _run_ex(B, layout, pol, ref, C, beta, gscale, normalize, nll_weight, pairs_total=0,
-            nll_tokens_total=0):
+            nll_tokens_total=0, reference_free=False):
     import torch
     dev = "cuda"
     t = lambda a: torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(dev)  # noqa: E731
@@ -21,10 +21,11 @@ def _run_ex(B, layout, pol, ref, C, beta, gscale, normalize, nll_weight, pairs_t
            [("loss", 1), ("acc", 1), ("m", B), ("cr", B), ("rr", B), ("w", B), ("coef", 2 * B),
             ("nll", 1)]}
     clen = torch.from_numpy(np.asarray(C, np.int32)).to(dev)
-    libdpo.loss_ex(B, layout, t(pol), t(ref), beta, gscale, out["loss"], out["acc"], out["m"],
-                   out["cr"], out["rr"], out["w"], out["coef"], out["nll"], normalize=normalize,
-                   nll_weight=nll_weight, completion_len=clen, pairs_total=pairs_total,
-                   nll_tokens_total=nll_tokens_total)
+    libdpo.loss_ex(B, layout, t(pol), None if ref is None else t(ref), beta, gscale, out["loss"],
+                   out["acc"], out["m"], out["cr"], out["rr"], out["w"], out["coef"], out["nll"],
+                   normalize=normalize, nll_weight=nll_weight, completion_len=clen,
+                   pairs_total=pairs_total, nll_tokens_total=nll_tokens_total,
+                   reference_free=reference_free)
     return {k: np64(v) for k, v in out.items()}
 
 
@@ -103,3 +104,50 @@ def test_data_parallel_shares_against_the_oracle(normalize, nll):
     assert abs(tot[0] - whole["loss"]) <= TOL_LOSS
     assert tot[1] == pytest.approx(whole["accuracy"], abs=1e-6)
     assert abs(tot[2] - whole["nll"]) <= 1e-5 * max(1.0, abs(whole["nll"]))
+
+
+@pytest.mark.parametrize("layout", ["halves", "adjacent"])
+@pytest.mark.parametrize("normalize,nll", [(False, 0.0), (True, 0.0), (True, 0.5)])
+def test_reference_free_on_identical_sums(layout, normalize, nll):
+    """reference_free against the oracle's reference-free loss (ref=None); a reference
+    buffer full of NaN passed beside the flag must not be read."""
+    rng = np.random.default_rng(74)
+    for B in (1, 5, 300):
+        C = rng.integers(1, 600, 2 * B)
+        pol = (-rng.uniform(0.01, 0.05, 2 * B) * C).astype(np.float32)
+        o = O.dpo_loss(pol.astype(np.float64), None, 0.1, layout, grad_scale=0.5,
+                       completion_len=C, normalize=normalize, nll_weight=nll)
+        nan_ref = np.full(2 * B, np.nan, np.float32)
+        for ref in (None, nan_ref):
+            g = _run_ex(B, layout, pol, ref, C, 0.1, 0.5, normalize, nll, reference_free=True)
+            assert abs(g["loss"][0] - o["loss"]) <= TOL_LOSS
+            assert g["acc"][0] == pytest.approx(o["accuracy"], abs=1e-7)
+            np.testing.assert_allclose(g["m"], o["margins"], rtol=1e-5, atol=1e-6)
+            np.testing.assert_allclose(g["cr"], o["chosen_rewards"], rtol=1e-5, atol=1e-6)
+            np.testing.assert_allclose(g["rr"], o["rejected_rewards"], rtol=1e-5, atol=1e-6)
+            np.testing.assert_allclose(g["w"], o["weights"], rtol=1e-5, atol=1e-7)
+            np.testing.assert_allclose(g["coef"], o["row_coef"], rtol=1e-5, atol=1e-10)
+
+
+def test_reference_free_end_to_end_through_the_backward():
+    """No reference forward at all: policy sums -> reference-free loss -> backward, against
+    the oracle's pipeline on the same inputs."""
+    import torch
+    w = WL.make_custom(R=6, L=160, d=128, V=900, dtype="bf16", seed=75, prompt_range=(1, 60),
+                       min_completion=1)
+    dw = DeviceWorkload(w)
+    H = WL.widen(w.H, "bf16")
+    Wd = WL.widen(w.W, "bf16")
+    op = O.seq_logprobs(H, Wd, w.tokens, w.prompt_len, w.completion_len)
+    ol = O.dpo_loss(op["seq_logp"], None, w.beta, w.layout)
+    pol, _, lse = dw.forward(dw.W, want_grad=True)
+    B = w.R // 2
+    out = {k: torch.empty(n, device="cuda") for k, n in [("loss", 1), ("coef", 2 * B)]}
+    libdpo.loss_ex(B, w.layout, pol, None, w.beta, 1.0, out["loss"], row_coef=out["coef"],
+                   reference_free=True)
+    assert abs(out["loss"].item() - ol["loss"]) <= TOL_LOSS
+    dH, dW = dw.backward(lse, out["coef"])
+    assert libdpo.check() == libdpo.OK
+    oH, oW = O.backward(H, Wd, w.tokens, w.prompt_len, w.completion_len, ol["row_coef"])
+    assert rel_frob(np64(dH), oH) <= TOL_GRAD
+    assert rel_frob(np64(dW), oW) <= TOL_GRAD
