@@ -159,7 +159,11 @@ dpo_status dpo_loss(int32_t B, int32_t layout, const float* pol, const float* re
  *                   reference model; the pages give no formula): the reference sums
  *                   are read as 0, so rewards are beta * pi (normalised when asked)
  *                   and the margin beta * (pi_c - pi_r); ref is not read and may be
- *                   NULL. Composes with the options above. */
+ *                   NULL. Composes with the options above.
+ * Zero-initialise the struct (dpo_loss_options o = {0};) and set the fields wanted: zero
+ * is "off" for every field. The struct grew with reference_free (library version 0.3.0);
+ * a caller built against an older header passes a shorter struct, so check
+ * dpo_version() >= 300 before relying on this layout. */
 typedef struct {
   int32_t normalize;
   float nll_weight;
