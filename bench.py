@@ -43,11 +43,10 @@ CONFIG_TEXT = ("Llama-3.1-8B head shape: 4 pairs -> 8 rows, seq 2048, prompt U{2
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
-def dh_launches(Nc, d, V, pairs=74):
-    """Kernel launches of the library's dH = dz.W for Nc positions (its plan, restated for
-    the launch count): one launch over the vocabulary (in chunks of 2^20 columns beyond
-    that), or one launch split over the vocabulary into K parts plus one reduce kernel
-    when the parts fill the rounds of 74 CTA pairs better by the plan's estimate."""
+def dh_parts(Nc, d, V, pairs=74):
+    """K parts of the library's dH = dz.W for Nc positions (its plan, restated for the
+    launch count): 1, or the vocabulary split into parts of one launch when they fill the
+    rounds of 74 CTA pairs better by the plan's estimate (0 when there is nothing to do)."""
     kb = -(-V // 64)
     tiles = -(-Nc // 256) * -(-d // 256)
     if tiles == 0:
@@ -67,6 +66,15 @@ def dh_launches(Nc, d, V, pairs=74):
         e = est(tiles * n, kbp) * (1.0 + 0.02 * (n - 1))
         if e < best * 0.97:
             best, parts = e, n
+    return parts
+
+
+def dh_launches(Nc, d, V):
+    """Kernel launches of the library's dH: one split launch plus its reduce kernel, or one
+    launch over the vocabulary (in chunks of 2^20 columns beyond that)."""
+    parts = dh_parts(Nc, d, V)
+    if parts == 0:
+        return 0
     return 2 if parts > 1 else -(-V // (1 << 20))
 
 

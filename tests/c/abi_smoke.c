@@ -115,7 +115,26 @@ static int gpu_step(void) {
   CHECK(fabsf(loss - (float)log(2.0)) < 1e-6f);
   CHECK(acc == 0.0f && wts[0] == 0.5f && wts[1] == 0.5f);
   for (int r = 0; r < R; ++r) CHECK(pol[r] < 0.0f && pol[r] > -20.0f * C[r]);
-  printf("gpu step ok: loss %.7f, sums %.3f %.3f %.3f %.3f\n", loss, pol[0], pol[1], pol[2], pol[3]);
+
+  /* reference-free objective: no reference buffer at all, the same bits as a reference of
+     zeros through dpo_loss */
+  float loss_free, loss_zero;
+  dpo_loss_options opt = {0};
+  opt.reference_free = 1;
+  CHECK(dpo_loss_ex(B, DPO_PAIRS_HALVES, (float*)dpol, NULL, 0.1f, 1.0f, &opt, (float*)dloss,
+                    NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL) == DPO_OK);
+  cudaMemcpy(&loss_free, dloss, 4, cudaMemcpyDeviceToHost);
+  CHECK(cudaMemset(dref, 0, sizeof(float) * R) == cudaSuccess);
+  CHECK(dpo_loss(B, DPO_PAIRS_HALVES, (float*)dpol, (float*)dref, 0.1f, 1.0f, (float*)dloss, NULL,
+                 NULL, NULL, NULL, NULL, NULL, NULL) == DPO_OK);
+  cudaMemcpy(&loss_zero, dloss, 4, cudaMemcpyDeviceToHost);
+  CHECK(loss_free == loss_zero);
+  opt.reference_free = 0;
+  CHECK(dpo_loss_ex(B, DPO_PAIRS_HALVES, (float*)dpol, NULL, 0.1f, 1.0f, &opt, (float*)dloss,
+                    NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL) == DPO_ERR_INVALID_ARG);
+  CHECK(dpo_check(NULL) == DPO_OK);
+  printf("gpu step ok: loss %.7f, sums %.3f %.3f %.3f %.3f, reference-free loss %.7f\n", loss,
+         pol[0], pol[1], pol[2], pol[3], loss_free);
   return 0;
 }
 

@@ -295,7 +295,7 @@ def test_dh_split_plan_matches_the_bench_launch_count(lib, R, L, d, V):
         libdpo.set_gemm_variant(old)
     nc = int(C.sum())
     split = bw_split > bw_plain
-    assert (bench.dh_launches(nc, d, V) == 2) == split    # one split launch + its reduce
+    assert (bench.dh_parts(nc, d, V) > 1) == split        # one split launch + its reduce
     if split:                                             # >= one part's fp32 partial sums
         assert bw_split - bw_plain >= nc * d * 4
 
