@@ -454,7 +454,9 @@ def run_ours(args):
     def step(timed=None):
         step_with(bp, br, timed)
 
-    def step_with(bp, br, timed=None):
+    def step_with(bp, br, timed=None, ref_sums=None):
+        """One step; with ref_sums (stored reference sums) the reference forward is
+        skipped, as in training on offline-scored reference log-probs."""
         if fwd_only:
             if timed is not None:
                 ev[0].record(stream)
@@ -469,10 +471,12 @@ def run_ours(args):
         libdpo.seq_logprobs(bp, True, pol, None, lse, ws, stream=sp)
         if timed is not None:
             ev[1].record(stream)
-        libdpo.seq_logprobs(br, False, ref, None, None, ws, stream=sp)
+        if ref_sums is None:
+            libdpo.seq_logprobs(br, False, ref, None, None, ws, stream=sp)
         if timed is not None:
             ev[2].record(stream)
-        libdpo.loss_ex(B, w.layout, pol, ref, w.beta, 1.0, outs["loss"], outs["accuracy"],
+        libdpo.loss_ex(B, w.layout, pol, ref if ref_sums is None else ref_sums, w.beta, 1.0,
+                       outs["loss"], outs["accuracy"],
                        outs["margins"], outs["cr"], outs["rr"], outs["w"], outs["coef"],
                        pairs_total=pairs_total, stream=sp)
         if timed is not None:
@@ -560,6 +564,28 @@ def run_ours(args):
     st = libdpo.check(sp)
     if st != libdpo.OK:
         raise RuntimeError(f"device status after timing: {libdpo.status_string(st)}")
+
+    # ------------------------------------------------------------ offline-scored reference
+    # The same step with the reference sums read from storage instead of a reference
+    # forward (the reference scored once, offline): policy forward, loss, backward.
+    offline_ms = None
+    if not fwd_only:
+        ref_stored = ref.clone()
+        for _ in range(2):
+            step_with(bp, br, ref_sums=ref_stored)
+        if ws_n > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        o0 = torch.cuda.Event(enable_timing=True)
+        o1 = torch.cuda.Event(enable_timing=True)
+        o0.record(stream)
+        for _ in range(args.steps):
+            step_with(bp, br, ref_sums=ref_stored)
+        o1.record(stream)
+        torch.cuda.synchronize(dev)
+        if ws_n > 1:
+            dist.barrier()
+        offline_ms = o0.elapsed_time(o1)
 
     # ------------------------------------------------------------ end to end (host buffers)
     # Every step uploads its inputs (H, tokens) from pinned host memory and reads its
@@ -657,7 +683,8 @@ def run_ours(args):
 
     # ------------------------------------------------------------ aggregate over ranks
     # each repetition's time is the max over ranks; the median repetition is reported
-    t = torch.tensor(rep_ms + e2e_reps + [float(Nc)], device=dev, dtype=torch.float64)
+    t = torch.tensor(rep_ms + e2e_reps + [offline_ms or 0.0, float(Nc)], device=dev,
+                     dtype=torch.float64)
     if ws_n > 1:
         tmax = t.clone()
         dist.all_reduce(tmax, op=dist.ReduceOp.MAX)
@@ -665,6 +692,8 @@ def run_ours(args):
         dist.all_reduce(tsum, op=dist.ReduceOp.SUM)
         rep_ms = [float(x) for x in tmax[:args.reps]]
         e2e_reps = [float(x) for x in tmax[args.reps:2 * args.reps]]
+        if offline_ms is not None:
+            offline_ms = float(tmax[-2])
         total_nc = float(tsum[-1])
     else:
         total_nc = float(Nc)
@@ -743,6 +772,14 @@ def run_ours(args):
             },
             "cpu_baseline": cpu,
             "cublas_same_box": cublas,
+            "offline_reference_step": None if offline_ms is None else {
+                "ms_per_step": offline_ms / args.steps,
+                "value": total_nc * args.steps / (offline_ms / 1e3), "unit": UNIT,
+                "gemms_per_step": 4,
+                "pct_of_peak_executed": 4 * gemm_flop * args.steps / (offline_ms / 1e3) / 1e12
+                                        / sustained,
+                "note": "policy forward + loss on stored reference sums + backward (reference "
+                        "scored offline); one timed loop right after the main repetitions"},
             "logits_mean_metric": {"ms": lm_ms, "bytes": lm_bytes,
                                    "GB/s": lm_bytes / (lm_ms / 1e3) / 1e9,
                                    "frac": lm_bytes / (lm_ms / 1e3) / 1e9 / hbm_peak,
