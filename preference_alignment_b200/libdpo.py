@@ -77,14 +77,20 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
 
 
 def _ptr(x) -> Optional[int]:
-    """Device/host address of a torch tensor, numpy array or raw integer; None -> NULL."""
+    """Device/host address of a torch tensor, numpy array or raw integer; None -> NULL.
+    The C ABI reads dense row-major arrays, so a strided view (a transpose, a column
+    slice) is refused rather than passed as its first element's address."""
     if x is None:
         return None
     if isinstance(x, int):
         return x
     if hasattr(x, "data_ptr"):
+        if x.numel() > 0 and not x.is_contiguous():
+            raise ValueError(f"tensor of shape {tuple(x.shape)} is not contiguous")
         return x.data_ptr()
     if isinstance(x, np.ndarray):
+        if not x.flags["C_CONTIGUOUS"]:
+            raise ValueError(f"array of shape {x.shape} is not C-contiguous")
         return x.ctypes.data
     raise TypeError(f"cannot take the address of {type(x)}")
 

@@ -348,3 +348,15 @@ def test_ipc_calls_fail_cleanly_without_device_memory(lib):
     with pytest.raises(libdpo.DpoError) as e:
         libdpo.ipc_close(0)
     assert e.value.status == libdpo.ERR_INVALID_ARG
+
+
+def test_binding_refuses_strided_views(lib):
+    """The C ABI reads dense arrays: a transposed or column-sliced device buffer is refused
+    by the binding instead of being passed as the address of its first element (host row
+    tables are copied to dense int32 arrays by BatchArgs)."""
+    import torch
+    dense = torch.zeros(2, 4)
+    with pytest.raises(ValueError):
+        libdpo.loss(2, "halves", dense.t(), FAKE, 0.1, 1.0, FAKE)
+    with pytest.raises(ValueError):
+        libdpo.loss(2, "halves", FAKE, FAKE, 0.1, 1.0, FAKE, margins=torch.zeros(2, 2)[:, 0])
