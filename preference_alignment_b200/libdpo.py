@@ -76,23 +76,38 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     return lib
 
 
-def _ptr(x) -> Optional[int]:
+# element types a buffer argument may have (bf16 data may also arrive as its 16-bit pattern)
+_KINDS = {"f32": ("float32",), "i32": ("int32",), "f16": ("float16",),
+          "bf16": ("bfloat16", "int16", "uint16")}
+
+
+def _ptr(x, kind: Optional[str] = None) -> Optional[int]:
     """Device/host address of a torch tensor, numpy array or raw integer; None -> NULL.
-    The C ABI reads dense row-major arrays, so a strided view (a transpose, a column
-    slice) is refused rather than passed as its first element's address."""
+    The C ABI reads dense row-major arrays of the element type its header names, so a
+    strided view (a transpose, a column slice) or a tensor of another element type
+    (`kind`: "f32", "i32", "bf16") is refused rather than passed on; a raw integer
+    address is taken as it is."""
     if x is None:
         return None
     if isinstance(x, int):
         return x
     if hasattr(x, "data_ptr"):
-        if x.numel() > 0 and not x.is_contiguous():
-            raise ValueError(f"tensor of shape {tuple(x.shape)} is not contiguous")
-        return x.data_ptr()
-    if isinstance(x, np.ndarray):
-        if not x.flags["C_CONTIGUOUS"]:
-            raise ValueError(f"array of shape {x.shape} is not C-contiguous")
-        return x.ctypes.data
-    raise TypeError(f"cannot take the address of {type(x)}")
+        name = str(x.dtype).replace("torch.", "")
+        ptr = x.data_ptr()
+        dense = x.numel() == 0 or x.is_contiguous()
+        shape = tuple(x.shape)
+    elif isinstance(x, np.ndarray):
+        name = x.dtype.name
+        ptr = x.ctypes.data
+        dense = bool(x.flags["C_CONTIGUOUS"])
+        shape = x.shape
+    else:
+        raise TypeError(f"cannot take the address of {type(x)}")
+    if not dense:
+        raise ValueError(f"buffer of shape {shape} is not contiguous")
+    if kind is not None and name not in _KINDS[kind]:
+        raise TypeError(f"expected a {kind} buffer, got {name} (shape {shape})")
+    return ptr
 
 
 def _stream(s) -> Optional[int]:
@@ -126,6 +141,9 @@ def set_wait_budget_ms(ms: int) -> int:
     return load().dpo_set_wait_budget_ms(int(ms))
 
 
+_HW_KIND = {BF16: "bf16", F32: "f32", F16: "f16"}
+
+
 class BatchArgs:
     """A dpo_batch plus the Python objects its pointers refer to (kept alive)."""
 
@@ -140,8 +158,10 @@ class BatchArgs:
         d = d if d is not None else shapeH[2]
         V = V if V is not None else shapeW[0]
         self.keep = (H, W, tokens)
-        self.c = Batch(int(R), int(L), int(d), int(V), DTYPES.get(dtype, dtype) if isinstance(dtype, str) else int(dtype),
-                       _ptr(H), _ptr(W), _ptr(tokens), self.prompt_len.ctypes.data,
+        self.dtype = DTYPES.get(dtype, dtype) if isinstance(dtype, str) else int(dtype)
+        self.c = Batch(int(R), int(L), int(d), int(V), self.dtype,
+                       _ptr(H, _HW_KIND.get(self.dtype)), _ptr(W, _HW_KIND.get(self.dtype)),
+                       _ptr(tokens, "i32"), self.prompt_len.ctypes.data,
                        self.completion_len.ctypes.data)
 
     @property
@@ -167,8 +187,9 @@ def _nbytes(ws, ws_bytes):
 
 def seq_logprobs(batch: BatchArgs, want_grad: bool, seq_logp, tok_logp, lse_state, ws,
                  ws_bytes=None, stream=None):
-    _check(load().dpo_seq_logprobs(ctypes.byref(batch.c), 1 if want_grad else 0, _ptr(seq_logp),
-                                   _ptr(tok_logp), _ptr(lse_state), _ptr(ws), _nbytes(ws, ws_bytes),
+    _check(load().dpo_seq_logprobs(ctypes.byref(batch.c), 1 if want_grad else 0,
+                                   _ptr(seq_logp, "f32"), _ptr(tok_logp, "f32"),
+                                   _ptr(lse_state, "f32"), _ptr(ws), _nbytes(ws, ws_bytes),
                                    _stream(stream)), "dpo_seq_logprobs")
 
 
@@ -176,9 +197,11 @@ def loss(B: int, layout, pol, ref, beta: float, grad_scale: float, loss_out, acc
          margins=None, chosen_rewards=None, rejected_rewards=None, weights=None, row_coef=None,
          stream=None):
     lay = LAYOUTS[layout] if isinstance(layout, str) else int(layout)
-    _check(load().dpo_loss(int(B), lay, _ptr(pol), _ptr(ref), float(beta), float(grad_scale),
-                           _ptr(loss_out), _ptr(accuracy), _ptr(margins), _ptr(chosen_rewards),
-                           _ptr(rejected_rewards), _ptr(weights), _ptr(row_coef), _stream(stream)),
+    _check(load().dpo_loss(int(B), lay, _ptr(pol, "f32"), _ptr(ref, "f32"), float(beta),
+                           float(grad_scale), _ptr(loss_out, "f32"), _ptr(accuracy, "f32"),
+                           _ptr(margins, "f32"), _ptr(chosen_rewards, "f32"),
+                           _ptr(rejected_rewards, "f32"), _ptr(weights, "f32"),
+                           _ptr(row_coef, "f32"), _stream(stream)),
            "dpo_loss")
 
 
@@ -202,19 +225,21 @@ def loss_ex(B: int, layout, pol, ref, beta: float, grad_scale: float, loss_out, 
     fn.argtypes = [ctypes.c_int32, ctypes.c_int32, vp, vp, ctypes.c_float, ctypes.c_float,
                    ctypes.POINTER(LossOptions), vp, vp, vp, vp, vp, vp, vp, vp, vp]
     fn.restype = ctypes.c_int
-    opt = LossOptions(1 if normalize else 0, float(nll_weight), _ptr(completion_len),
+    opt = LossOptions(1 if normalize else 0, float(nll_weight), _ptr(completion_len, "i32"),
                       int(pairs_total), int(nll_tokens_total), 1 if reference_free else 0)
     lay = LAYOUTS[layout] if isinstance(layout, str) else int(layout)
-    _check(fn(int(B), lay, _ptr(pol), _ptr(ref), float(beta), float(grad_scale), ctypes.byref(opt),
-              _ptr(loss_out), _ptr(accuracy), _ptr(margins), _ptr(chosen_rewards),
-              _ptr(rejected_rewards), _ptr(weights), _ptr(row_coef), _ptr(nll), _stream(stream)),
+    _check(fn(int(B), lay, _ptr(pol, "f32"), _ptr(ref, "f32"), float(beta), float(grad_scale),
+              ctypes.byref(opt), _ptr(loss_out, "f32"), _ptr(accuracy, "f32"), _ptr(margins, "f32"),
+              _ptr(chosen_rewards, "f32"), _ptr(rejected_rewards, "f32"), _ptr(weights, "f32"),
+              _ptr(row_coef, "f32"), _ptr(nll, "f32"), _stream(stream)),
            "dpo_loss_ex")
 
 
 def backward(batch: BatchArgs, lse_state, row_coef, dH, dW, accumulate_dW: bool, ws,
              ws_bytes=None, stream=None):
-    _check(load().dpo_backward(ctypes.byref(batch.c), _ptr(lse_state), _ptr(row_coef), _ptr(dH),
-                               _ptr(dW), 1 if accumulate_dW else 0, _ptr(ws),
+    _check(load().dpo_backward(ctypes.byref(batch.c), _ptr(lse_state, "f32"),
+                               _ptr(row_coef, "f32"), _ptr(dH, "f32"), _ptr(dW, "f32"),
+                               1 if accumulate_dW else 0, _ptr(ws),
                                _nbytes(ws, ws_bytes), _stream(stream)), "dpo_backward")
 
 
@@ -228,7 +253,7 @@ def backward_dw(batch: BatchArgs, v_begin: int, v_end: int, dW, accumulate_dW: b
     fn.argtypes = [ctypes.POINTER(Batch), ctypes.c_int32, ctypes.c_int32, vp, ctypes.c_int,
                    ctypes.c_int32, vp, ctypes.c_size_t, vp]
     fn.restype = ctypes.c_int
-    _check(fn(ctypes.byref(batch.c), int(v_begin), int(v_end), _ptr(dW),
+    _check(fn(ctypes.byref(batch.c), int(v_begin), int(v_end), _ptr(dW, "f32"),
               1 if accumulate_dW else 0, int(max_sms), _ptr(ws), _nbytes(ws, ws_bytes),
               _stream(stream)), "dpo_backward_dw")
 
@@ -240,7 +265,7 @@ def backward_dh(batch: BatchArgs, dH, ws, ws_bytes=None, max_sms: int = 0, strea
     vp = ctypes.c_void_p
     fn.argtypes = [ctypes.POINTER(Batch), vp, ctypes.c_int32, vp, ctypes.c_size_t, vp]
     fn.restype = ctypes.c_int
-    _check(fn(ctypes.byref(batch.c), _ptr(dH), int(max_sms), _ptr(ws), _nbytes(ws, ws_bytes),
+    _check(fn(ctypes.byref(batch.c), _ptr(dH, "f32"), int(max_sms), _ptr(ws), _nbytes(ws, ws_bytes),
               _stream(stream)), "dpo_backward_dh")
 
 
@@ -263,7 +288,7 @@ def backward_dw_scatter(batch: BatchArgs, n_ranks: int, rank: int, rows_per_rank
     fn.argtypes = [ctypes.POINTER(Batch), ctypes.POINTER(DwScatter), ctypes.c_int32, vp,
                    ctypes.c_size_t, vp]
     fn.restype = ctypes.c_int
-    ptrs = [_ptr(r) for r in recv]
+    ptrs = [_ptr(r, "f32") for r in recv]
     if len(ptrs) != n_ranks or n_ranks > MAX_SCATTER_RANKS:
         raise ValueError("recv needs one buffer per rank (at most 8 ranks)")
     x = DwScatter(int(n_ranks), int(rank), int(rows_per_rank),
@@ -280,7 +305,8 @@ def dw_reduce_slots(recv, n_slots: int, rows: int, d: int, dW_shard, accumulate:
     vp = ctypes.c_void_p
     fn.argtypes = [vp, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, vp, ctypes.c_int, vp]
     fn.restype = ctypes.c_int
-    _check(fn(_ptr(recv), int(n_slots), int(rows), int(d), _ptr(dW_shard), 1 if accumulate else 0,
+    _check(fn(_ptr(recv, "f32"), int(n_slots), int(rows), int(d), _ptr(dW_shard, "f32"),
+              1 if accumulate else 0,
               _stream(stream)), "dpo_dw_reduce_slots")
 
 
@@ -332,7 +358,8 @@ def shard_logprob_parts(batch: BatchArgs, offset: int, total: int, shard_lse, sh
     fn.argtypes = [ctypes.POINTER(Batch), ctypes.POINTER(VocabShard), vp, vp, vp, ctypes.c_size_t, vp]
     fn.restype = ctypes.c_int
     sh = VocabShard(int(offset), int(total))
-    _check(fn(ctypes.byref(batch.c), ctypes.byref(sh), _ptr(shard_lse), _ptr(shard_zy), _ptr(ws),
+    _check(fn(ctypes.byref(batch.c), ctypes.byref(sh), _ptr(shard_lse, "f32"),
+              _ptr(shard_zy, "f32"), _ptr(ws),
               _nbytes(ws, ws_bytes), _stream(stream)), "dpo_shard_logprob_parts")
 
 
@@ -345,8 +372,9 @@ def shard_combine(batch: BatchArgs, total: int, n_shards: int, shard_lse, shard_
     fn.argtypes = [ctypes.POINTER(Batch), ctypes.c_int32, ctypes.c_int32, vp, vp, vp, vp, vp, vp,
                    ctypes.c_size_t, vp]
     fn.restype = ctypes.c_int
-    _check(fn(ctypes.byref(batch.c), int(total), int(n_shards), _ptr(shard_lse), _ptr(shard_zy),
-              _ptr(seq_logp), _ptr(tok_logp), _ptr(lse_state), _ptr(ws), _nbytes(ws, ws_bytes),
+    _check(fn(ctypes.byref(batch.c), int(total), int(n_shards), _ptr(shard_lse, "f32"),
+              _ptr(shard_zy, "f32"), _ptr(seq_logp, "f32"), _ptr(tok_logp, "f32"),
+              _ptr(lse_state, "f32"), _ptr(ws), _nbytes(ws, ws_bytes),
               _stream(stream)), "dpo_shard_combine")
 
 
@@ -360,8 +388,9 @@ def shard_backward(batch: BatchArgs, offset: int, total: int, lse_state, row_coe
                    vp, ctypes.c_size_t, vp]
     fn.restype = ctypes.c_int
     sh = VocabShard(int(offset), int(total))
-    _check(fn(ctypes.byref(batch.c), ctypes.byref(sh), _ptr(lse_state), _ptr(row_coef),
-              _ptr(dH_part), _ptr(dW_shard), 1 if accumulate_dW else 0, _ptr(ws),
+    _check(fn(ctypes.byref(batch.c), ctypes.byref(sh), _ptr(lse_state, "f32"),
+              _ptr(row_coef, "f32"), _ptr(dH_part, "f32"), _ptr(dW_shard, "f32"),
+              1 if accumulate_dW else 0, _ptr(ws),
               _nbytes(ws, ws_bytes), _stream(stream)), "dpo_shard_backward")
 
 
@@ -374,7 +403,7 @@ def logits_mean(batch: BatchArgs, layout, means, ws, ws_bytes=None, stream=None)
                    ctypes.c_size_t, ctypes.c_void_p]
     fn.restype = ctypes.c_int
     lay = LAYOUTS[layout] if isinstance(layout, str) else int(layout)
-    _check(fn(ctypes.byref(batch.c), lay, _ptr(means), _ptr(ws), _nbytes(ws, ws_bytes),
+    _check(fn(ctypes.byref(batch.c), lay, _ptr(means, "f32"), _ptr(ws), _nbytes(ws, ws_bytes),
               _stream(stream)), "dpo_logits_mean")
 
 
@@ -425,8 +454,9 @@ def seq_logprobs_noalloc(batch: BatchArgs, want_grad: bool, seq_logp, tok_logp, 
     fn.argtypes = [ctypes.POINTER(Batch), ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
                    ctypes.c_void_p, ctypes.c_void_p]
     fn.restype = ctypes.c_int
-    _check(fn(ctypes.byref(batch.c), 1 if want_grad else 0, _ptr(seq_logp), _ptr(tok_logp),
-              _ptr(lse_state), _stream(stream)), "dpo_seq_logprobs_noalloc")
+    _check(fn(ctypes.byref(batch.c), 1 if want_grad else 0, _ptr(seq_logp, "f32"),
+              _ptr(tok_logp, "f32"), _ptr(lse_state, "f32"), _stream(stream)),
+           "dpo_seq_logprobs_noalloc")
 
 
 NOALLOC_SCRATCH_BYTES = 32 << 20

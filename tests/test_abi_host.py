@@ -360,3 +360,20 @@ def test_binding_refuses_strided_views(lib):
         libdpo.loss(2, "halves", dense.t(), FAKE, 0.1, 1.0, FAKE)
     with pytest.raises(ValueError):
         libdpo.loss(2, "halves", FAKE, FAKE, 0.1, 1.0, FAKE, margins=torch.zeros(2, 2)[:, 0])
+
+
+def test_binding_refuses_buffers_of_another_element_type(lib):
+    """Outputs the header declares fp32 refuse fp64 tensors, tokens refuse int64, and the
+    bf16 batch refuses fp32 weights, before any call into the library."""
+    import torch
+    with pytest.raises(TypeError):
+        libdpo.loss(2, "halves", FAKE, FAKE, 0.1, 1.0, torch.zeros(1, dtype=torch.float64))
+    with pytest.raises(TypeError):
+        libdpo.BatchArgs(FAKE, FAKE, torch.zeros(4, 8, dtype=torch.int64), np.ones(4, np.int32),
+                         np.ones(4, np.int32), R=4, L=8, d=8, V=8)
+    with pytest.raises(TypeError):
+        libdpo.BatchArgs(FAKE, torch.zeros(8, 8), FAKE, np.ones(4, np.int32), np.ones(4, np.int32),
+                         R=4, L=8, d=8, V=8, dtype="bf16")
+    b = libdpo.BatchArgs(FAKE, torch.zeros(8, 8, dtype=torch.bfloat16), FAKE, np.ones(4, np.int32),
+                         np.ones(4, np.int32), R=4, L=8, d=8, V=8, dtype="bf16")
+    assert b.c.V == 8
