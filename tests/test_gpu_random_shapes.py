@@ -59,3 +59,40 @@ def test_random_shape_against_the_oracle(R, L, d, V, dtype, layout, seed):
     oH, oW = O.backward(H, Wd, w.tokens, w.prompt_len, w.completion_len, ol["row_coef"])
     assert rel_frob(np64(dH), oH) <= TOL_GRAD
     assert rel_frob(np64(dW), oW) <= TOL_GRAD
+
+
+@pytest.mark.parametrize("R,L,d,V,dtype,layout,seed", _cases(n=16, seed=20261204))
+def test_random_shape_chunked_backward_and_vocab_shards(R, L, d, V, dtype, layout, seed):
+    """The same comparison through the smallest backward workspace (token chunks of 128
+    whenever there are more scored positions) and through the vocabulary-parallel calls
+    over 1 to 4 shards run one after the other."""
+    import torch
+    from preference_alignment_b200.vp import shard_range
+    from test_gpu_vocab_shards import _sharded_backward, _sharded_forward
+    w = WL.make_custom(R=R, L=L, d=d, V=V, dtype=dtype, layout=layout, seed=seed,
+                       ref_std=0.05)
+    dw = DeviceWorkload(w)
+    H = WL.widen(w.H, dtype)
+    Wd = WL.widen(w.W, dtype)
+    op = O.seq_logprobs(H, Wd, w.tokens, w.prompt_len, w.completion_len)
+    coef_np = np.random.default_rng(seed).normal(0.0, 0.05, R)
+    oH, oW = O.backward(H, Wd, w.tokens, w.prompt_len, w.completion_len, coef_np)
+    coef = torch.from_numpy(coef_np.astype(np.float32)).cuda()
+
+    _, _, lse = dw.forward(dw.W, want_grad=True)
+    _, _, mn = libdpo.workspace_size(dw.batch())
+    dH, dW = dw.backward(lse, coef, ws_bytes=mn)
+    assert libdpo.check() == libdpo.OK
+    assert rel_frob(np64(dH), oH) <= TOL_GRAD
+    assert rel_frob(np64(dW), oW) <= TOL_GRAD
+
+    n = min(V, 1 + seed % 4)
+    shards = [shard_range(V, n, k) for k in range(n)]
+    seq, tok, lse_s, _, _ = _sharded_forward(dw, shards)
+    assert libdpo.check() == libdpo.OK
+    assert np.abs(np64(tok) - op["tok_logp"]).max(initial=0.0) <= TOL_TOK
+    assert_seq_close(np64(seq), op["seq_logp"])
+    dHs, dWs = _sharded_backward(dw, shards, lse_s, coef)
+    assert libdpo.check() == libdpo.OK
+    assert rel_frob(np64(dHs), oH) <= TOL_GRAD
+    assert rel_frob(np64(dWs), oW) <= TOL_GRAD
